@@ -1,0 +1,105 @@
+"""Python side of the fp64 CPU oracle (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this module.  The product package never does.
+
+``attention_rows`` wraps ``varlen_oracle.c`` (built with gcc into
+``liboracle_varlen.so`` next to this file).  That C file is the plain
+definition of the packed attention forward pass of boostr 0.2.0
+varlen_attention.rs (VarLenAttentionOps, "Layout contract") computed per
+(token, head) row in fp64, following realizar 0.8.4 attention.rs IMP-111
+(standard_single_head_attention / standard_softmax); see its header for the
+readings taken where the pages are silent.
+
+``schedule`` (in ``oracle/schedule.py``) is the CPU statement of the tile
+work list the GPU scheduler must reproduce bit-exactly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "varlen_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle_varlen.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (no CUDA involved)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        fn = lib.oracle_varlen_attention_rows
+        fn.restype = ctypes.c_int
+        fn.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 + [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        _lib = lib
+    return _lib
+
+
+def _bits(x) -> np.ndarray:
+    """bf16 tensor / uint16 array -> contiguous uint16 numpy array of bit patterns."""
+    if hasattr(x, "dtype") and str(getattr(x, "dtype")) == "torch.bfloat16":
+        import torch
+        x = x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint16:
+        raise TypeError("oracle inputs must be bf16 tensors or uint16 bit-pattern arrays")
+    return x
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def attention_rows(q, k, v, cu_q: Sequence[int], cu_k: Sequence[int], H: int, H_kv: int,
+                   D: int, causal: bool, window: int = 0,
+                   rows: Optional[np.ndarray] = None, nthreads: Optional[int] = None):
+    """fp64 output rows and logsumexp.
+
+    q: [total_q, H, D] bf16; k, v: [total_k, H_kv, D] bf16 (torch bf16 or uint16 bits).
+    rows: optional int array [n, 2] of (token, head) pairs; None = all rows.
+    Returns (out [n, D] float64, lse [n] float64); with rows=None, shaped
+    [total_q, H, D] and [total_q, H].
+    """
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    cq = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int32))
+    ck = np.ascontiguousarray(np.asarray(cu_k, dtype=np.int32))
+    batch = len(cq) - 1
+    total_q = int(cq[-1])
+    if rows is None:
+        n = total_q * H
+        tok_p = head_p = None
+    else:
+        rows = np.asarray(rows)
+        tok = np.ascontiguousarray(rows[:, 0].astype(np.int64))
+        hd = np.ascontiguousarray(rows[:, 1].astype(np.int32))
+        n = len(tok)
+        tok_p, head_p = tok.ctypes.data, hd.ctypes.data
+    out = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    rc = lib.oracle_varlen_attention_rows(
+        qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, cq.ctypes.data, ck.ctypes.data,
+        batch, H, H_kv, D, int(bool(causal)), int(window), tok_p, head_p, n,
+        out.ctypes.data, lse.ctypes.data, int(nthreads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_varlen_attention_rows failed with code {rc}")
+    if rows is None:
+        return out.reshape(total_q, H, D), lse.reshape(total_q, H)
+    return out, lse

@@ -1,0 +1,194 @@
+/*
+ * Plain fp64 CPU oracle for the variable-length packed attention forward pass.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg load this library.  The CUDA product path
+ * never links, calls or includes anything from this directory, and this file
+ * includes nothing from the product.
+ *
+ * What it computes (per query token t and query head h), following
+ *   - boostr 0.2.0 varlen_attention.rs, VarLenAttentionOps docs,
+ *     "Layout contract", "GQA key/value head mapping", "Cumulative sequence
+ *     lengths": q [total_q, H, D], k/v [total_k, H_kv, D], sequence b owns
+ *     query rows cu_q[b]..cu_q[b+1]-1 and key rows cu_k[b]..cu_k[b+1]-1;
+ *     kv_head = h / (H / H_kv); output [total_q, H, D]; logsumexp [total_q, H];
+ *   - realizar 0.8.4 attention.rs, IMP-111 standard_single_head_attention and
+ *     standard_softmax: scores = q.k * (1/sqrt(D)), softmax(x) =
+ *     exp(x - max) / sum exp(x - max), output = softmax(scores) @ V;
+ *   - boostr flash.rs FlashAttentionOps docs, "Sliding window": with
+ *     window_size W > 0 a query sees only the W most recent key positions;
+ *     logsumexp is F32 and is what the backward pass consumes.
+ *
+ * Readings taken where the pages are silent (each one is listed in the
+ * design notes of this repository):
+ *   - causal with L_q != L_k is bottom-right aligned: key j is visible to
+ *     query i iff j <= i + (L_k - L_q);
+ *   - the window holds exactly W keys ending at the diagonal:
+ *     i + delta - W + 1 <= j <= i + delta, and W > 0 implies the upper bound
+ *     even without the causal flag;
+ *   - logsumexp is the natural log of sum_j exp(s_ij) over the visible keys
+ *     of the SCALED scores s_ij = q_i.k_j / sqrt(D);
+ *   - a query with no visible key gets output 0 and logsumexp -inf.
+ *
+ * Inputs are bf16 bit patterns; each is widened exactly to double.  All
+ * arithmetic is double.  Rows are independent, so threads split the list of
+ * requested (token, head) rows; nothing is blocked, fused or reordered
+ * inside a row.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double bf16_bits_to_double(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Sequence b owning packed query token t: the b with cu_q[b] <= t < cu_q[b+1]. */
+static int owning_sequence(const int32_t* cu_q, int batch, int64_t t) {
+    int lo = 0, hi = batch - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) / 2;
+        if ((int64_t)cu_q[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+/* The visibility predicate, written out as stated above. */
+static int key_visible(int64_t i, int64_t j, int64_t L_q, int64_t L_k,
+                       int causal, int window) {
+    int64_t delta = L_k - L_q;
+    if (j < 0 || j >= L_k) return 0;
+    if (causal && j > i + delta) return 0;
+    if (window > 0) {
+        if (j > i + delta) return 0;
+        if (j < i + delta - window + 1) return 0;
+    }
+    return 1;
+}
+
+typedef struct {
+    const uint16_t *q, *k, *v;
+    const int32_t *cu_q, *cu_k;
+    int batch, H, H_kv, D, causal, window;
+    const int64_t* row_token; /* NULL => all rows r = t*H + h */
+    const int32_t* row_head;
+    int64_t row_begin, row_end;
+    double* out; /* [n_rows, D] */
+    double* lse; /* [n_rows] */
+    int64_t max_lk;
+} job_t;
+
+static void one_row(const job_t* jb, int64_t r, double* s) {
+    int64_t t;
+    int h;
+    if (jb->row_token) { t = jb->row_token[r]; h = jb->row_head[r]; }
+    else { t = r / jb->H; h = (int)(r % jb->H); }
+    const int D = jb->D;
+    const int b = owning_sequence(jb->cu_q, jb->batch, t);
+    const int64_t L_q = (int64_t)jb->cu_q[b + 1] - jb->cu_q[b];
+    const int64_t L_k = (int64_t)jb->cu_k[b + 1] - jb->cu_k[b];
+    const int64_t i = t - jb->cu_q[b];
+    const int group = jb->H / jb->H_kv;
+    const int hk = h / group;
+    const double scale = 1.0 / sqrt((double)D);
+    const uint16_t* qrow = jb->q + ((size_t)t * jb->H + h) * D;
+    double* o = jb->out + (size_t)r * D;
+
+    /* scores of the visible keys; s[j] = -inf marks an invisible key */
+    double m = -INFINITY;
+    int64_t n_vis = 0;
+    for (int64_t j = 0; j < L_k; ++j) {
+        if (!key_visible(i, j, L_q, L_k, jb->causal, jb->window)) { s[j] = -INFINITY; continue; }
+        const uint16_t* krow = jb->k + (((size_t)jb->cu_k[b] + j) * jb->H_kv + hk) * D;
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += bf16_bits_to_double(qrow[d]) * bf16_bits_to_double(krow[d]);
+        s[j] = dot * scale;
+        if (s[j] > m) m = s[j];
+        ++n_vis;
+    }
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    if (n_vis == 0) { jb->lse[r] = -INFINITY; return; }
+
+    double l = 0.0;
+    for (int64_t j = 0; j < L_k; ++j) {
+        if (s[j] == -INFINITY) continue;
+        const double p = exp(s[j] - m);
+        l += p;
+        const uint16_t* vrow = jb->v + (((size_t)jb->cu_k[b] + j) * jb->H_kv + hk) * D;
+        for (int d = 0; d < D; ++d) o[d] += p * bf16_bits_to_double(vrow[d]);
+    }
+    for (int d = 0; d < D; ++d) o[d] /= l;
+    jb->lse[r] = m + log(l);
+}
+
+static void* run_job(void* arg) {
+    const job_t* jb = (const job_t*)arg;
+    double* s = (double*)malloc(sizeof(double) * (size_t)(jb->max_lk > 0 ? jb->max_lk : 1));
+    if (!s) return (void*)1;
+    for (int64_t r = jb->row_begin; r < jb->row_end; ++r) one_row(jb, r, s);
+    free(s);
+    return NULL;
+}
+
+/*
+ * Compute output and logsumexp rows in fp64.
+ *
+ * q, k, v:     bf16 bit patterns, packed [total_q, H, D] and [total_k, H_kv, D].
+ * cu_q, cu_k:  host int32 [batch + 1] cumulative lengths.
+ * row_token, row_head: optional (token, head) pairs to compute (n_rows of
+ *              them); when row_token is NULL every row is computed in the
+ *              order r = token * H + head and n_rows must be total_q * H.
+ * out:         [n_rows, D] doubles; lse: [n_rows] doubles.
+ * Returns 0, or -1 on an argument error, -2 on an allocation failure.
+ */
+int oracle_varlen_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                 const int32_t* cu_q, const int32_t* cu_k, int batch,
+                                 int H, int H_kv, int D, int causal, int window,
+                                 const int64_t* row_token, const int32_t* row_head,
+                                 int64_t n_rows, double* out, double* lse, int nthreads) {
+    if (batch < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || D < 1 || window < 0) return -1;
+    if (n_rows < 0 || (n_rows > 0 && (!out || !lse))) return -1;
+    if (!row_token && n_rows != (int64_t)cu_q[batch] * H) return -1;
+    if (row_token && !row_head) return -1;
+    int64_t max_lk = 0;
+    for (int b = 0; b < batch; ++b) {
+        int64_t lk = (int64_t)cu_k[b + 1] - cu_k[b];
+        if (lk > max_lk) max_lk = lk;
+    }
+    if (nthreads < 1) nthreads = 1;
+    if ((int64_t)nthreads > n_rows) nthreads = n_rows > 0 ? (int)n_rows : 1;
+
+    job_t* jobs = (job_t*)calloc((size_t)nthreads, sizeof(job_t));
+    pthread_t* tids = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !tids) { free(jobs); free(tids); return -2; }
+    int rc = 0;
+    for (int w = 0; w < nthreads; ++w) {
+        job_t* jb = &jobs[w];
+        jb->q = q; jb->k = k; jb->v = v; jb->cu_q = cu_q; jb->cu_k = cu_k;
+        jb->batch = batch; jb->H = H; jb->H_kv = H_kv; jb->D = D;
+        jb->causal = causal; jb->window = window;
+        jb->row_token = row_token; jb->row_head = row_head;
+        jb->row_begin = n_rows * w / nthreads;
+        jb->row_end = n_rows * (w + 1) / nthreads;
+        jb->out = out; jb->lse = lse; jb->max_lk = max_lk;
+    }
+    int started = 0;
+    for (int w = 1; w < nthreads; ++w) {
+        if (pthread_create(&tids[w], NULL, run_job, &jobs[w]) != 0) { rc = -2; break; }
+        started = w;
+    }
+    if (run_job(&jobs[0]) != NULL) rc = -2;
+    for (int w = 1; w <= started; ++w) {
+        void* ret = NULL;
+        pthread_join(tids[w], &ret);
+        if (ret != NULL) rc = -2;
+    }
+    free(jobs);
+    free(tids);
+    return rc;
+}
