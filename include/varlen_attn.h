@@ -1,0 +1,139 @@
+/*
+ * varlen_attn.h — C ABI of the B200 (sm_100a) packed variable-length
+ * attention forward pass.
+ *
+ * The operation is VarLenAttentionOps::varlen_attention_fwd of boostr 0.2.0
+ * (src/ops/traits/attention/varlen_attention.rs), "Layout contract":
+ *   q   [total_q, num_heads,    head_dim]  bf16, packed queries
+ *   k   [total_k, num_kv_heads, head_dim]  bf16, packed keys
+ *   v   [total_k, num_kv_heads, head_dim]  bf16, packed values
+ *   cu_seqlens_q / cu_seqlens_k  int32 [batch + 1], "Cumulative sequence
+ *       lengths": cu[0] = 0, cu[i] = sum of the first i lengths; lengths
+ *       [512, 300, 128] give [0, 512, 812, 940]
+ *   out [total_q, num_heads, head_dim]  bf16
+ *   lse [total_q, num_heads]            f32, natural-log logsumexp
+ * "GQA key/value head mapping": kv_head = q_head / (num_heads / num_kv_heads),
+ * num_heads % num_kv_heads == 0; K/V are never repeated in memory.
+ * Scores are scaled by 1/sqrt(head_dim).  `causal` masks key j of query i
+ * when j > i + (L_k - L_q) (bottom-right alignment; for L_q == L_k this is
+ * j > i).  `window` > 0 keeps only the `window` most recent keys up to and
+ * including the diagonal (boostr flash.rs, FlashAttentionOps docs, "Sliding
+ * window"); 0 disables it.  A query with no visible key gets out = 0 and
+ * lse = -inf.  lse is ln sum_j exp(q.k_j / sqrt(head_dim)) over the visible
+ * keys (the quantity the backward pass of the same trait consumes).
+ *
+ * Memory and ownership: every pointer of varlen_attention_fwd is device
+ * memory owned by the caller; nothing is retained after the call returns.
+ * q, k, v, out must be 16-byte aligned, contiguous, row-major as above.  The
+ * library allocates its workspace stream-ordered (cudaMallocAsync /
+ * cudaFreeAsync on `stream`) and frees it on the same stream.
+ *
+ * Asynchrony: the call only enqueues work on `stream` (a cudaStream_t,
+ * NULL = the legacy default stream) and never synchronises; cu_seqlens stay
+ * on the device.  Launch errors are returned; device-side conditions (a
+ * bounded barrier wait that gave up, more query tiles than max_seqlen_q
+ * allows for) set bits in a device status word read by
+ * varlen_attention_device_status().
+ *
+ * Preconditions not checked on the device: cu arrays are non-decreasing with
+ * cu[0] = 0; max_seqlen_q / max_seqlen_k are >= every L_q / L_k (they size
+ * the workspace and the tensor maps and are never used for indexing).
+ * Violations can give wrong results; out-of-range rows are not read (tiles
+ * past the end of the tensors are fetched with bounds-checked loads).
+ *
+ * Errors: each entry point returns VA_OK or a negative code and records a
+ * message retrievable with varlen_attention_last_error() (per host thread).
+ */
+#ifndef VARLEN_ATTN_H
+#define VARLEN_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VA_OK 0
+#define VA_ERR_INVALID_ARG (-1) /* null pointer, negative size, H % H_kv != 0, misalignment */
+#define VA_ERR_UNSUPPORTED (-2) /* head_dim other than 64 or 128, sizes beyond int32 indexing */
+#define VA_ERR_CUDA (-3)        /* a CUDA runtime / driver call or a launch failed */
+
+/* Device status bits (varlen_attention_device_status). */
+#define VA_STATUS_WAIT_TIMEOUT 1u       /* a bounded wait inside a kernel gave up */
+#define VA_STATUS_SCHEDULE_OVERFLOW 2u  /* more query tiles than max_seqlen_q allows for */
+
+/* Path selection for varlen_attention_fwd_ex. */
+#define VA_PATH_AUTO 0    /* decode when max_seqlen_q == 1, else prefill */
+#define VA_PATH_PREFILL 1 /* tensor-core tile kernel (any L_q) */
+#define VA_PATH_DECODE 2  /* split-K K/V streaming kernel (requires every L_q <= 1) */
+
+/*
+ * Packed variable-length attention forward (see the file comment).
+ * Argument order follows VarLenAttentionOps::varlen_attention_fwd of boostr
+ * 0.2.0 varlen_attention.rs, with `window` (FlashAttentionOps "Sliding
+ * window") added and the outputs passed in instead of returned.
+ * head_dim must be 64 or 128.  batch == 0 or max_seqlen_q == 0 is a no-op.
+ */
+int varlen_attention_fwd(const void* q, const void* k, const void* v,
+                         const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                         int batch, int num_heads, int num_kv_heads,
+                         int max_seqlen_q, int max_seqlen_k, int head_dim,
+                         int causal, int window, void* out, float* lse, void* stream);
+
+/*
+ * Same as varlen_attention_fwd with the path forced (VA_PATH_*) and, for the
+ * decode path, the number of keys per split (decode_split_keys in [32, 1024],
+ * 0 = library default).  Used by tests that check path and split invariance.
+ */
+int varlen_attention_fwd_ex(const void* q, const void* k, const void* v,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            int batch, int num_heads, int num_kv_heads,
+                            int max_seqlen_q, int max_seqlen_k, int head_dim,
+                            int causal, int window, void* out, float* lse,
+                            int path, int decode_split_keys, void* stream);
+
+/*
+ * End-to-end variant on HOST buffers: the same operation with q, k, v,
+ * cu_seqlens_q, cu_seqlens_k, out and lse all in host memory (pinned memory
+ * gives asynchronous copies; pageable memory works but is staged by CUDA).
+ * Copies inputs to the device, runs varlen_attention_fwd on `stream`, copies
+ * out and lse back and synchronises `stream` before returning.  Device
+ * buffers are allocated and freed stream-ordered inside the call.
+ */
+int varlen_attention_fwd_host(const void* q, const void* k, const void* v,
+                              const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                              int batch, int num_heads, int num_kv_heads,
+                              int max_seqlen_q, int max_seqlen_k, int head_dim,
+                              int causal, int window, void* out, float* lse, void* stream);
+
+/*
+ * The longest-first query-tile work list the prefill path builds from
+ * cu_seqlens (device pointers), written to `tiles` (device int32
+ * [capacity][4] = {sequence, query tile, first key tile, end key tile}) and
+ * its length to `n_tiles` (device int32).  Tiles hold 128 query rows and 128
+ * keys; key tiles [first, end) hold every key any row of the tile can see,
+ * end == first when none.  Order: descending end - first, ties by ascending
+ * (sequence, query tile).  capacity must be >= the number of query tiles,
+ * otherwise *n_tiles = 0 and VA_STATUS_SCHEDULE_OVERFLOW is raised.
+ */
+int varlen_attention_schedule(const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                              int batch, int max_seqlen_q, int causal, int window,
+                              int32_t* tiles, int32_t* n_tiles, int capacity, void* stream);
+
+/*
+ * Synchronise the current device, then store the device status word
+ * (VA_STATUS_* bits, 0 = clean) in *status and, if clear != 0, reset it.
+ */
+int varlen_attention_device_status(unsigned* status, int clear);
+
+/* Message for the last non-VA_OK return on this host thread ("" if none). */
+const char* varlen_attention_last_error(void);
+
+/* Library ABI version (major * 100 + minor). */
+int varlen_attention_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VARLEN_ATTN_H */

@@ -1,0 +1,65 @@
+"""Shared helpers for the parity tests: run the CUDA path and the oracle on
+the same seeded inputs and compare element by element."""
+import numpy as np
+import torch
+
+from variable_length_flash_varlen_b200 import binding, workloads
+
+O_TOL = 1e-2    # max |O_gpu - O_oracle|
+LSE_TOL = 1e-3  # max |LSE_gpu - LSE_oracle|
+
+
+def to_device_inputs(wl, q, k, v):
+    dev = "cuda"
+    cu_q = torch.tensor(wl.cu_q, dtype=torch.int32, device=dev)
+    cu_k = torch.tensor(wl.cu_k, dtype=torch.int32, device=dev)
+    return q.to(dev), k.to(dev), v.to(dev), cu_q, cu_k
+
+
+def run_gpu(wl, q, k, v, path=binding.VA_PATH_AUTO, split_keys=0, dev_inputs=None):
+    dq, dk, dv, cu_q, cu_k = dev_inputs or to_device_inputs(wl, q, k, v)
+    out = torch.full_like(dq, float("nan"))
+    lse = torch.full((dq.shape[0], wl.H), float("nan"), dtype=torch.float32, device="cuda")
+    binding.varlen_attention_fwd(dq, dk, dv, cu_q, cu_k, wl.batch, wl.H, wl.H_kv,
+                                 wl.max_seqlen_q, wl.max_seqlen_k, wl.D, wl.causal, wl.window,
+                                 out=out, lse=lse, path=path, decode_split_keys=split_keys)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def oracle_all(oracle_lib, wl, q, k, v):
+    return oracle_lib.attention_rows(q, k, v, wl.cu_q, wl.cu_k, wl.H, wl.H_kv, wl.D,
+                                     wl.causal, wl.window)
+
+
+def compare(out_gpu, lse_gpu, out_ref, lse_ref, rows=None):
+    """Element-wise comparison; returns (max |dO|, max |dLSE|)."""
+    o = out_gpu.float().cpu().double().numpy()
+    l = lse_gpu.float().cpu().double().numpy()
+    if rows is not None:
+        o = o[rows[:, 0], rows[:, 1]]
+        l = l[rows[:, 0], rows[:, 1]]
+    assert not np.isnan(o).any(), "NaN in GPU output"
+    assert not np.isnan(l).any(), "NaN in GPU logsumexp"
+    neg_ref = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(l), neg_ref), "-inf logsumexp rows differ"
+    d_o = float(np.max(np.abs(o - out_ref))) if o.size else 0.0
+    fin = ~neg_ref
+    d_l = float(np.max(np.abs(l[fin] - lse_ref[fin]))) if fin.any() else 0.0
+    assert d_o <= O_TOL, f"max |dO| = {d_o}"
+    assert d_l <= LSE_TOL, f"max |dLSE| = {d_l}"
+    return d_o, d_l
+
+
+def sample_rows(wl, n_random, seed=0):
+    """(token, head) rows: random ones plus the first and last row of every sequence."""
+    rng = np.random.default_rng(seed)
+    toks = [rng.integers(0, wl.total_q, n_random)]
+    edge = []
+    for b in range(wl.batch):
+        if wl.lengths_q[b] > 0:
+            edge += [wl.cu_q[b], wl.cu_q[b + 1] - 1]
+    toks.append(np.array(edge, dtype=np.int64))
+    t = np.concatenate(toks)
+    h = rng.integers(0, wl.H, len(t))
+    return np.stack([t, h], axis=1)

@@ -1,0 +1,77 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds, loads,
+exports every entry point include/varlen_attn.h declares, and rejects bad
+arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from variable_length_flash_varlen_b200 import binding, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "varlen_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(varlen_attention_\w+)\s*\(", text)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    assert "varlen_attention_fwd" in names
+    assert set(names) == set(binding.SIGNATURES), "binding and header disagree"
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.varlen_attention_version() == 100
+
+
+def _call(lib, **over):
+    a = dict(q=16, k=16, v=16, cq=16, ck=16, batch=1, H=4, Hkv=2, mq=8, mk=8, D=64,
+             causal=1, window=0, out=16, lse=16)
+    a.update(over)
+    return lib.varlen_attention_fwd(a["q"], a["k"], a["v"], a["cq"], a["ck"], a["batch"], a["H"],
+                                    a["Hkv"], a["mq"], a["mk"], a["D"], a["causal"], a["window"],
+                                    a["out"], a["lse"], None)
+
+
+@pytest.mark.parametrize("over,code,needle", [
+    (dict(H=4, Hkv=3), -1, "multiple"),
+    (dict(D=96), -2, "head_dim"),
+    (dict(batch=-1), -1, "batch"),
+    (dict(window=-2), -1, "window"),
+    (dict(Hkv=0), -1, "num_kv_heads"),
+    (dict(q=None), -1, "q is NULL"),
+    (dict(lse=None), -1, "lse is NULL"),
+    (dict(out=8), -1, "aligned"),
+    (dict(mq=-1), -1, "max_seqlen"),
+])
+def test_invalid_arguments_rejected_without_gpu(lib, over, code, needle):
+    rc = _call(lib, **over)
+    assert rc == code
+    assert needle in lib.varlen_attention_last_error().decode()
+
+
+def test_empty_batch_is_noop(lib):
+    assert _call(lib, batch=0, q=None, k=None, v=None, out=None, lse=None) == 0
+    assert _call(lib, mq=0, q=None, k=None, v=None, out=None, lse=None) == 0
+    assert lib.varlen_attention_last_error().decode() == ""
+
+
+def test_decode_split_keys_range_checked(lib):
+    f = lib.varlen_attention_fwd_ex
+    rc = f(16, 16, 16, 16, 16, 1, 4, 2, 8, 8, 64, 0, 0, 16, 16, 9, 0, None)
+    assert rc == -1 and "path" in lib.varlen_attention_last_error().decode()
+    rc = f(16, 16, 16, 16, 16, 1, 4, 2, 8, 8, 64, 0, 0, 16, 16, 2, 0, None)
+    assert rc == -1 and "max_seqlen_q" in lib.varlen_attention_last_error().decode()

@@ -1,0 +1,160 @@
+"""ctypes binding of ``libvarlen_attn.so`` (argument marshalling only).
+
+Every function here takes torch tensors, checks dtypes / shapes / devices and
+passes raw pointers to the C entry point of the same name declared in
+``include/varlen_attn.h``.  No arithmetic happens on the Python side and
+there is no fallback: if the library is missing, ``load()`` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvarlen_attn.so")
+
+VA_OK = 0
+VA_PATH_AUTO, VA_PATH_PREFILL, VA_PATH_DECODE = 0, 1, 2
+VA_STATUS_WAIT_TIMEOUT = 1
+VA_STATUS_SCHEDULE_OVERFLOW = 2
+
+# every symbol the header declares, with its ctypes signature
+_P, _I = ctypes.c_void_p, ctypes.c_int
+SIGNATURES = {
+    "varlen_attention_fwd": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
+    "varlen_attention_fwd_ex": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _I, _I, _P]),
+    "varlen_attention_fwd_host": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
+    "varlen_attention_schedule": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P]),
+    "varlen_attention_device_status": (_I, [ctypes.POINTER(ctypes.c_uint), _I]),
+    "varlen_attention_last_error": (ctypes.c_char_p, []),
+    "varlen_attention_version": (_I, []),
+}
+
+_lib = None
+
+
+class VarlenAttentionError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"{message} (code {code})")
+        self.code = code
+
+
+def load(path: Optional[str] = None):
+    """Load the in-tree library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise FileNotFoundError(
+            f"{p} is missing: build it with `python -m variable_length_flash_varlen_b200.build`")
+    lib = ctypes.CDLL(p)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _check(rc: int):
+    if rc != VA_OK:
+        raise VarlenAttentionError(rc, load().varlen_attention_last_error().decode())
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check_inputs(q, k, v, cu_q, cu_k, num_heads, num_kv_heads, head_dim, device_kind):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.device.type != device_kind:
+            raise ValueError(f"{name} must be on {device_kind}")
+    for name, t in (("cu_seqlens_q", cu_q), ("cu_seqlens_k", cu_k)):
+        if t.dtype != torch.int32 or not t.is_contiguous() or t.device.type != device_kind:
+            raise ValueError(f"{name} must be a contiguous int32 {device_kind} tensor")
+    if q.dim() != 3 or q.shape[1:] != (num_heads, head_dim):
+        raise ValueError("q must be [total_q, num_heads, head_dim]")
+    if k.shape != v.shape or k.dim() != 3 or k.shape[1:] != (num_kv_heads, head_dim):
+        raise ValueError("k and v must be [total_k, num_kv_heads, head_dim]")
+
+
+def varlen_attention_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                         cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                         batch: int, num_heads: int, num_kv_heads: int,
+                         max_seqlen_q: int, max_seqlen_k: int, head_dim: int,
+                         causal: bool, window: int = 0,
+                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                         stream: Optional[torch.cuda.Stream] = None,
+                         path: int = VA_PATH_AUTO, decode_split_keys: int = 0
+                         ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Packed attention forward on device tensors; returns (out, lse)."""
+    lib = load()
+    _check_inputs(q, k, v, cu_seqlens_q, cu_seqlens_k, num_heads, num_kv_heads, head_dim, "cuda")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[0], num_heads, dtype=torch.float32, device=q.device)
+    if out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    if lse.shape != (q.shape[0], num_heads) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [total_q, num_heads] tensor")
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens_q.data_ptr(),
+            cu_seqlens_k.data_ptr(), batch, num_heads, num_kv_heads, max_seqlen_q, max_seqlen_k,
+            head_dim, int(bool(causal)), int(window), out.data_ptr(), lse.data_ptr())
+    if path == VA_PATH_AUTO and decode_split_keys == 0:
+        rc = lib.varlen_attention_fwd(*args, _stream_ptr(stream))
+    else:
+        rc = lib.varlen_attention_fwd_ex(*args, int(path), int(decode_split_keys),
+                                         _stream_ptr(stream))
+    _check(rc)
+    return out, lse
+
+
+def varlen_attention_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                              cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                              batch: int, num_heads: int, num_kv_heads: int,
+                              max_seqlen_q: int, max_seqlen_k: int, head_dim: int,
+                              causal: bool, window: int, out: torch.Tensor, lse: torch.Tensor,
+                              stream: Optional[torch.cuda.Stream] = None):
+    """Same operation on host (ideally pinned) tensors; blocks until out/lse are filled."""
+    lib = load()
+    _check_inputs(q, k, v, cu_seqlens_q, cu_seqlens_k, num_heads, num_kv_heads, head_dim, "cpu")
+    if out.device.type != "cpu" or lse.device.type != "cpu":
+        raise ValueError("out and lse must be host tensors")
+    rc = lib.varlen_attention_fwd_host(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(),
+        batch, num_heads, num_kv_heads, max_seqlen_q, max_seqlen_k, head_dim, int(bool(causal)),
+        int(window), out.data_ptr(), lse.data_ptr(), _stream_ptr(stream))
+    _check(rc)
+    return out, lse
+
+
+def varlen_attention_schedule(cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor, batch: int,
+                              max_seqlen_q: int, causal: bool, window: int, capacity: int,
+                              stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """The device-built query-tile list as an int32 [n, 4] tensor (b, qt, kt_lo, kt_hi)."""
+    lib = load()
+    tiles = torch.zeros(capacity, 4, dtype=torch.int32, device=cu_seqlens_q.device)
+    n = torch.zeros(1, dtype=torch.int32, device=cu_seqlens_q.device)
+    _check(lib.varlen_attention_schedule(cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), batch,
+                                         max_seqlen_q, int(bool(causal)), int(window),
+                                         tiles.data_ptr(), n.data_ptr(), capacity,
+                                         _stream_ptr(stream)))
+    torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
+    return tiles[: int(n.item())]
+
+
+def device_status(clear: bool = True) -> int:
+    st = ctypes.c_uint(0)
+    _check(load().varlen_attention_device_status(ctypes.byref(st), int(clear)))
+    return st.value

@@ -1,0 +1,74 @@
+// Work list of query tiles, built on the device from cu_seqlens.
+//
+// Every sequence b's queries are cut into tiles of kBlockM rows; for each
+// tile the key tiles (kBlockN keys) that any of its rows can see form the
+// half-open range [kt_lo, kt_hi).  Key tiles outside the range are never
+// loaded: the causal triangle above the diagonal and the keys older than a
+// sliding window (boostr flash.rs, FlashAttentionOps docs, "Sliding window")
+// cost nothing.  The list is sorted longest first (descending kt_hi - kt_lo,
+// ties by ascending (b, query tile)) so a persistent grid starts with the
+// heaviest tiles and finishes with the light ones.
+#pragma once
+
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace va {
+
+constexpr int kBlockM = 128;   // query rows per tile
+constexpr int kBlockN = 128;   // keys per tile
+constexpr int kSortCapacity = 16384;  // query tiles sorted in shared memory
+
+struct TileEntry {
+    int b, qt, kt_lo, kt_hi;
+};
+
+// Visible key interval [lo, hi] of query row i (sequence-relative) under the
+// readings used throughout: delta = L_k - L_q aligns the causal diagonal to
+// the bottom-right, and a window of W > 0 keeps exactly the W keys ending at
+// the diagonal.  Empty when lo > hi.
+__host__ __device__ __forceinline__ void row_key_interval(int i, int L_q, int L_k, bool causal,
+                                                          int window, int& lo, int& hi) {
+    const int diag = i + (L_k - L_q);
+    hi = L_k - 1;
+    if (causal || window > 0) hi = diag < hi ? diag : hi;
+    lo = 0;
+    if (window > 0) {
+        const int w0 = diag - window + 1;
+        lo = w0 > 0 ? w0 : 0;
+    }
+}
+
+// Key-tile range of query tile qt.  The intervals of consecutive rows have
+// non-decreasing ends and overlap or touch, so the union over the tile is the
+// interval of its first non-empty row to its last row.
+__host__ __device__ __forceinline__ void tile_key_range(int qt, int L_q, int L_k, bool causal,
+                                                        int window, int& kt_lo, int& kt_hi) {
+    kt_lo = kt_hi = 0;
+    if (L_k <= 0) return;
+    const int first = qt * kBlockM;
+    const int last = min(L_q, first + kBlockM) - 1;
+    if (last < first) return;
+    // first row whose interval is non-empty: diag >= 0 when the band is bounded above
+    int r0 = first;
+    if (causal || window > 0) {
+        const int need = L_q - L_k;  // diag >= 0  <=>  i >= L_q - L_k
+        if (need > r0) r0 = need;
+    }
+    if (r0 > last) return;
+    int lo0, hi0, lo1, hi1;
+    row_key_interval(r0, L_q, L_k, causal, window, lo0, hi0);
+    row_key_interval(last, L_q, L_k, causal, window, lo1, hi1);
+    if (hi1 < lo0) return;
+    kt_lo = lo0 / kBlockN;
+    kt_hi = hi1 / kBlockN + 1;
+}
+
+// Workspace header written by the builder and read by the attention kernels.
+struct SchedHeader {
+    int n_tiles;  // number of valid entries in the sorted list
+    int pad[3];
+};
+
+}  // namespace va

@@ -1,0 +1,393 @@
+// Host side of the C ABI declared in include/varlen_attn.h: argument
+// validation, stream-ordered workspace, tensor maps and kernel launches.
+// The whole library is this one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <climits>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "decode.cuh"
+#include "prefill_sm100.cuh"
+#include "schedule_build.cuh"
+#include "varlen_attn.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(VA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define VA_CUDA(call)                                        \
+    do {                                                     \
+        cudaError_t e_ = (call);                             \
+        if (e_ != cudaSuccess) return cuda_fail(e_, #call);  \
+    } while (0)
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int device_setup(int& dev, DeviceInfo*& info) {
+    VA_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return fail(VA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    info = &g_dev[dev];
+    if (info->ready) return VA_OK;
+    cudaDeviceProp prop;
+    VA_CUDA(cudaGetDeviceProperties(&prop, dev));
+    if (prop.major != 10)
+        return fail(VA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                    dev, prop.major, prop.minor);
+    info->num_sms = prop.multiProcessorCount;
+    if (!g_encode) {
+        cudaDriverEntryPointQueryResult q;
+        void* fn = nullptr;
+        VA_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+        if (q != cudaDriverEntryPointSuccess || !fn)
+            return fail(VA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::PrefillSmem<64>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::PrefillSmem<128>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::build_schedule_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::kSortCapacity * 8));
+    info->ready = true;
+    return VA_OK;
+}
+
+// 2-D bf16 view [rows][cols] (cols contiguous), box 64 x 128, 128-byte swizzle.
+int make_tile_map(CUtensorMap* map, const void* base, long long cols, long long rows) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(VA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return VA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Args {
+    const void *q, *k, *v;
+    const int32_t *cu_q, *cu_k;
+    int batch, H, H_kv, max_q, max_k, D, causal, window;
+    void* out;
+    float* lse;
+};
+
+int validate(const Args& a) {
+    if (a.batch < 0) return fail(VA_ERR_INVALID_ARG, "batch must be >= 0 (got %d)", a.batch);
+    if (a.H < 1) return fail(VA_ERR_INVALID_ARG, "num_heads must be >= 1 (got %d)", a.H);
+    if (a.H_kv < 1) return fail(VA_ERR_INVALID_ARG, "num_kv_heads must be >= 1 (got %d)", a.H_kv);
+    if (a.H % a.H_kv != 0)
+        return fail(VA_ERR_INVALID_ARG, "num_heads (%d) must be a multiple of num_kv_heads (%d)",
+                    a.H, a.H_kv);
+    if (a.D != 64 && a.D != 128)
+        return fail(VA_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", a.D);
+    if (a.window < 0) return fail(VA_ERR_INVALID_ARG, "window must be >= 0 (got %d)", a.window);
+    if (a.max_q < 0 || a.max_k < 0)
+        return fail(VA_ERR_INVALID_ARG, "max_seqlen_q/k must be >= 0 (got %d, %d)", a.max_q, a.max_k);
+    if (a.batch == 0 || a.max_q == 0) return VA_OK;
+    const char* names[] = {"q", "k", "v", "cu_seqlens_q", "cu_seqlens_k", "out", "lse"};
+    const void* ptrs[] = {a.q, a.k, a.v, a.cu_q, a.cu_k, a.out, a.lse};
+    for (int i = 0; i < 7; ++i)
+        if (!ptrs[i]) return fail(VA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+    if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.out))
+        return fail(VA_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(a.lse) & 3u) return fail(VA_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+    const long long rows_q = static_cast<long long>(a.batch) * a.max_q;
+    const long long rows_k = static_cast<long long>(a.batch) * a.max_k;
+    if (rows_q * a.H * (long long)a.D >= (1ll << 40) || rows_k * a.H_kv * (long long)a.D >= (1ll << 40))
+        return fail(VA_ERR_UNSUPPORTED, "tensors beyond 2^40 elements");
+    return VA_OK;
+}
+
+int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
+    const long long tiles_per_seq = (a.max_q + va::kBlockM - 1) / va::kBlockM;
+    const long long cap_ll = tiles_per_seq * a.batch;
+    if (cap_ll * a.H >= INT_MAX) return fail(VA_ERR_UNSUPPORTED, "too many query tiles x heads");
+    const int cap = static_cast<int>(cap_ll);
+    int key_slots = 1;
+    while (key_slots < cap && key_slots < va::kSortCapacity) key_slots <<= 1;
+
+    const size_t hdr_bytes = 256;
+    const size_t list_bytes = static_cast<size_t>(cap) * sizeof(va::TileEntry);
+    char* ws = nullptr;
+    VA_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&ws), hdr_bytes + 2 * list_bytes, stream));
+    auto* hdr = reinterpret_cast<va::SchedHeader*>(ws);
+    auto* scratch = reinterpret_cast<va::TileEntry*>(ws + hdr_bytes);
+    auto* tiles = reinterpret_cast<va::TileEntry*>(ws + hdr_bytes + list_bytes);
+
+    int rc = VA_OK;
+    CUtensorMap tq, tk, tv;
+    const long long rows_q = std::max(1ll, static_cast<long long>(a.batch) * a.max_q);
+    const long long rows_k = std::max(1ll, static_cast<long long>(a.batch) * a.max_k);
+    if ((rc = make_tile_map(&tq, a.q, static_cast<long long>(a.H) * a.D, rows_q)) != VA_OK ||
+        (rc = make_tile_map(&tk, a.k, static_cast<long long>(a.H_kv) * a.D, rows_k)) != VA_OK ||
+        (rc = make_tile_map(&tv, a.v, static_cast<long long>(a.H_kv) * a.D, rows_k)) != VA_OK) {
+        cudaFreeAsync(ws, stream);
+        return rc;
+    }
+
+    va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
+        a.cu_q, a.cu_k, a.batch, a.causal, a.window, cap, key_slots, scratch, tiles, hdr);
+    cudaError_t be = cudaGetLastError();
+    if (be != cudaSuccess) {
+        cudaFreeAsync(ws, stream);
+        return cuda_fail(be, "schedule build launch");
+    }
+
+    va::PrefillParams p;
+    p.cu_q = a.cu_q;
+    p.cu_k = a.cu_k;
+    p.batch = a.batch;
+    p.H = a.H;
+    p.H_kv = a.H_kv;
+    p.causal = a.causal;
+    p.window = a.window;
+    p.tiles = tiles;
+    p.hdr = hdr;
+    p.tile_capacity = cap;
+    p.q = static_cast<const __nv_bfloat16*>(a.q);
+    p.k = static_cast<const __nv_bfloat16*>(a.k);
+    p.v = static_cast<const __nv_bfloat16*>(a.v);
+    p.out = static_cast<__nv_bfloat16*>(a.out);
+    p.lse = a.lse;
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)));
+    const long long items = cap_ll * a.H;
+    const int grid = static_cast<int>(std::min<long long>(dev.num_sms, items));
+    if (a.D == 64)
+        va::prefill_fwd_kernel<64><<<grid, va::kPrefillThreads, va::PrefillSmem<64>::kAlloc, stream>>>(tq, tk, tv, p);
+    else
+        va::prefill_fwd_kernel<128><<<grid, va::kPrefillThreads, va::PrefillSmem<128>::kAlloc, stream>>>(tq, tk, tv, p);
+    cudaError_t le = cudaGetLastError();
+    cudaFreeAsync(ws, stream);
+    if (le != cudaSuccess) return cuda_fail(le, "prefill launch");
+    return VA_OK;
+}
+
+int run_decode(const Args& a, int split_keys, cudaStream_t stream) {
+    int chunk = split_keys > 0 ? split_keys : va::kDecodeMaxChunk;
+    if (chunk < 32 || chunk > va::kDecodeMaxChunk)
+        return fail(VA_ERR_INVALID_ARG, "decode_split_keys must be in [32, %d] (got %d)",
+                    va::kDecodeMaxChunk, split_keys);
+    const int n_split_max = std::max(1, (a.max_k + chunk - 1) / chunk);
+    const int G = a.H / a.H_kv;
+    const int groups = a.H_kv * ((G + va::kDecodeHeads - 1) / va::kDecodeHeads);
+    if (groups > 65535 || n_split_max > 65535)
+        return fail(VA_ERR_UNSUPPORTED, "decode grid too large (kv groups %d, splits %d)", groups,
+                    n_split_max);
+    const size_t slots = static_cast<size_t>(a.batch) * a.H * n_split_max;
+    char* ws = nullptr;
+    const size_t o_bytes = slots * a.D * sizeof(float);
+    VA_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&ws), o_bytes + slots * 2 * sizeof(float), stream));
+
+    va::DecodeParams p;
+    p.cu_q = a.cu_q;
+    p.cu_k = a.cu_k;
+    p.batch = a.batch;
+    p.H = a.H;
+    p.H_kv = a.H_kv;
+    p.causal = a.causal;
+    p.window = a.window;
+    p.q = static_cast<const __nv_bfloat16*>(a.q);
+    p.k = static_cast<const __nv_bfloat16*>(a.k);
+    p.v = static_cast<const __nv_bfloat16*>(a.v);
+    p.part_o = reinterpret_cast<float*>(ws);
+    p.part_ml = reinterpret_cast<float*>(ws + o_bytes);
+    p.n_split_max = n_split_max;
+    p.chunk = chunk;
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)));
+    p.out = static_cast<__nv_bfloat16*>(a.out);
+    p.lse = a.lse;
+    dim3 grid(a.batch, groups, n_split_max);
+    if (a.D == 64) {
+        va::decode_split_kernel<64><<<grid, va::kDecodeThreads, 0, stream>>>(p);
+        va::decode_combine_kernel<64><<<a.batch * a.H, 64, 0, stream>>>(p);
+    } else {
+        va::decode_split_kernel<128><<<grid, va::kDecodeThreads, 0, stream>>>(p);
+        va::decode_combine_kernel<128><<<a.batch * a.H, 128, 0, stream>>>(p);
+    }
+    cudaError_t le = cudaGetLastError();
+    cudaFreeAsync(ws, stream);
+    if (le != cudaSuccess) return cuda_fail(le, "decode launch");
+    return VA_OK;
+}
+
+int forward(const Args& a, int path, int split_keys, cudaStream_t stream) {
+    int rc = validate(a);
+    if (rc != VA_OK) return rc;
+    if (path != VA_PATH_AUTO && path != VA_PATH_PREFILL && path != VA_PATH_DECODE)
+        return fail(VA_ERR_INVALID_ARG, "unknown path %d", path);
+    if (a.batch == 0 || a.max_q == 0) return VA_OK;
+    if (path == VA_PATH_AUTO) path = a.max_q == 1 ? VA_PATH_DECODE : VA_PATH_PREFILL;
+    if (path == VA_PATH_DECODE && a.max_q > 1)
+        return fail(VA_ERR_INVALID_ARG, "the decode path needs max_seqlen_q <= 1 (got %d)", a.max_q);
+    if (static_cast<long long>(a.batch) * a.H > INT_MAX)
+        return fail(VA_ERR_UNSUPPORTED, "batch x num_heads beyond int32");
+    int dev;
+    DeviceInfo* info;
+    if ((rc = device_setup(dev, info)) != VA_OK) return rc;
+    return path == VA_PATH_DECODE ? run_decode(a, split_keys, stream) : run_prefill(a, *info, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int varlen_attention_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                         const int32_t* cu_seqlens_k, int batch, int num_heads, int num_kv_heads,
+                         int max_seqlen_q, int max_seqlen_k, int head_dim, int causal, int window,
+                         void* out, float* lse, void* stream) {
+    g_last_error[0] = 0;
+    Args a{q, k, v, cu_seqlens_q, cu_seqlens_k, batch, num_heads, num_kv_heads, max_seqlen_q,
+           max_seqlen_k, head_dim, causal ? 1 : 0, window, out, lse};
+    return forward(a, VA_PATH_AUTO, 0, static_cast<cudaStream_t>(stream));
+}
+
+int varlen_attention_fwd_ex(const void* q, const void* k, const void* v,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                            int num_heads, int num_kv_heads, int max_seqlen_q, int max_seqlen_k,
+                            int head_dim, int causal, int window, void* out, float* lse, int path,
+                            int decode_split_keys, void* stream) {
+    g_last_error[0] = 0;
+    Args a{q, k, v, cu_seqlens_q, cu_seqlens_k, batch, num_heads, num_kv_heads, max_seqlen_q,
+           max_seqlen_k, head_dim, causal ? 1 : 0, window, out, lse};
+    return forward(a, path, decode_split_keys, static_cast<cudaStream_t>(stream));
+}
+
+int varlen_attention_fwd_host(const void* q, const void* k, const void* v,
+                              const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                              int num_heads, int num_kv_heads, int max_seqlen_q, int max_seqlen_k,
+                              int head_dim, int causal, int window, void* out, float* lse,
+                              void* stream_) {
+    g_last_error[0] = 0;
+    Args a{q, k, v, cu_seqlens_q, cu_seqlens_k, batch, num_heads, num_kv_heads, max_seqlen_q,
+           max_seqlen_k, head_dim, causal ? 1 : 0, window, out, lse};
+    int rc = validate(a);
+    if (rc != VA_OK) return rc;
+    if (batch == 0 || max_seqlen_q == 0) return VA_OK;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const long long T_q = cu_seqlens_q[batch], T_k = cu_seqlens_k[batch];
+    if (T_q < 0 || T_k < 0) return fail(VA_ERR_INVALID_ARG, "negative total length");
+    const size_t qb = static_cast<size_t>(T_q) * num_heads * head_dim * 2;
+    const size_t kb = static_cast<size_t>(T_k) * num_kv_heads * head_dim * 2;
+    const size_t cb = static_cast<size_t>(batch + 1) * 4;
+    const size_t ob = qb, lb = static_cast<size_t>(T_q) * num_heads * 4;
+    auto up16 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    const size_t total = up16(qb) + 2 * up16(kb) + 2 * up16(cb) + up16(ob) + up16(lb);
+    char* ws = nullptr;
+    VA_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&ws), total, stream));
+    char* p = ws;
+    void* dq = p; p += up16(qb);
+    void* dk = p; p += up16(kb);
+    void* dv = p; p += up16(kb);
+    int32_t* dcq = reinterpret_cast<int32_t*>(p); p += up16(cb);
+    int32_t* dck = reinterpret_cast<int32_t*>(p); p += up16(cb);
+    void* dout = p; p += up16(ob);
+    float* dlse = reinterpret_cast<float*>(p);
+    cudaError_t e = cudaSuccess;
+    if (qb) e = cudaMemcpyAsync(dq, q, qb, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess && kb) e = cudaMemcpyAsync(dk, k, kb, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess && kb) e = cudaMemcpyAsync(dv, v, kb, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dcq, cu_seqlens_q, cb, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dck, cu_seqlens_k, cb, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) {
+        cudaFreeAsync(ws, stream);
+        return cuda_fail(e, "host-to-device copy");
+    }
+    Args d{dq, dk, dv, dcq, dck, batch, num_heads, num_kv_heads, max_seqlen_q, max_seqlen_k,
+           head_dim, causal ? 1 : 0, window, dout, dlse};
+    rc = forward(d, VA_PATH_AUTO, 0, stream);
+    if (rc == VA_OK && ob) e = cudaMemcpyAsync(out, dout, ob, cudaMemcpyDeviceToHost, stream);
+    if (rc == VA_OK && e == cudaSuccess && lb)
+        e = cudaMemcpyAsync(lse, dlse, lb, cudaMemcpyDeviceToHost, stream);
+    cudaFreeAsync(ws, stream);
+    cudaError_t se = cudaStreamSynchronize(stream);
+    if (rc != VA_OK) return rc;
+    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+    if (se != cudaSuccess) return cuda_fail(se, "cudaStreamSynchronize");
+    return VA_OK;
+}
+
+int varlen_attention_schedule(const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                              int max_seqlen_q, int causal, int window, int32_t* tiles,
+                              int32_t* n_tiles, int capacity, void* stream_) {
+    g_last_error[0] = 0;
+    if (batch < 1) return fail(VA_ERR_INVALID_ARG, "batch must be >= 1 (got %d)", batch);
+    if (!cu_seqlens_q || !cu_seqlens_k || !tiles || !n_tiles)
+        return fail(VA_ERR_INVALID_ARG, "NULL pointer argument");
+    if (capacity < 1 || window < 0 || max_seqlen_q < 0)
+        return fail(VA_ERR_INVALID_ARG, "capacity must be >= 1, window and max_seqlen_q >= 0");
+    if (reinterpret_cast<uintptr_t>(tiles) & 15u) return fail(VA_ERR_INVALID_ARG, "tiles must be 16-byte aligned");
+    int dev;
+    DeviceInfo* info;
+    int rc = device_setup(dev, info);
+    if (rc != VA_OK) return rc;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    int key_slots = 1;
+    while (key_slots < capacity && key_slots < va::kSortCapacity) key_slots <<= 1;
+    char* ws = nullptr;
+    const size_t list_bytes = static_cast<size_t>(capacity) * sizeof(va::TileEntry);
+    VA_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&ws), 256 + list_bytes, stream));
+    auto* hdr = reinterpret_cast<va::SchedHeader*>(ws);
+    va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
+        cu_seqlens_q, cu_seqlens_k, batch, causal ? 1 : 0, window, capacity, key_slots,
+        reinterpret_cast<va::TileEntry*>(ws + 256), reinterpret_cast<va::TileEntry*>(tiles), hdr);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(n_tiles, &hdr->n_tiles, sizeof(int32_t), cudaMemcpyDeviceToDevice, stream);
+    cudaFreeAsync(ws, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "schedule build");
+    return VA_OK;
+}
+
+int varlen_attention_device_status(unsigned* status, int clear) {
+    g_last_error[0] = 0;
+    if (!status) return fail(VA_ERR_INVALID_ARG, "status is NULL");
+    VA_CUDA(cudaDeviceSynchronize());
+    VA_CUDA(cudaMemcpyFromSymbol(status, va::g_va_status, sizeof(unsigned)));
+    if (clear) {
+        const unsigned zero = 0;
+        VA_CUDA(cudaMemcpyToSymbol(va::g_va_status, &zero, sizeof(unsigned)));
+    }
+    return VA_OK;
+}
+
+const char* varlen_attention_last_error(void) { return g_last_error; }
+
+int varlen_attention_version(void) { return 100; }
+
+}  // extern "C"
