@@ -118,8 +118,10 @@ decode_split_kernel(const DecodeParams p) {
         }
     }
 
-    // ---- scores: one row group per key, D/8 lanes per row
-    for (int base = grp; base < n; base += NGRP * kDecodeUnroll) {
+    // ---- scores: one row group per key, D/8 lanes per row.  The trip count
+    // is the same for every lane (warp shuffles below need the whole warp).
+    for (int base0 = 0; base0 < n; base0 += NGRP * kDecodeUnroll) {
+        const int base = base0 + grp;
         uint4 kr[kDecodeUnroll];
 #pragma unroll
         for (int u = 0; u < kDecodeUnroll; ++u) {
@@ -182,7 +184,8 @@ decode_split_kernel(const DecodeParams p) {
     for (int g = 0; g < kDecodeHeads; ++g)
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
-    for (int base = grp; base < n; base += NGRP * kDecodeUnroll) {
+    for (int base0 = 0; base0 < n; base0 += NGRP * kDecodeUnroll) {
+        const int base = base0 + grp;
         uint4 vr[kDecodeUnroll];
 #pragma unroll
         for (int u = 0; u < kDecodeUnroll; ++u) {

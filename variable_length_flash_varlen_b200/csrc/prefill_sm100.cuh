@@ -175,7 +175,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const TileEntry te = p.tiles[idx / p.H];
             const int h = idx % p.H, hk = h / group;
             if (te.kt_hi <= te.kt_lo) continue;
-            if (!(ok = mbar_wait(q_empty, (q_issued & 1) ^ 1, abort_flag, &g_va_status))) break;
+            if (!(ok = mbar_wait_warp(q_empty, (q_issued & 1) ^ 1, abort_flag, &g_va_status))) break;
             load_tile<D>(smem + L::kQ, &tmQ, p.q, p.cu_q[te.b] + te.qt * kBlockM, T_q, q_stride,
                          h * D, q_full, lane);
             ++q_issued;
@@ -183,11 +183,11 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             for (int kt = te.kt_lo; kt < te.kt_hi; ++kt) {
                 const int s = k_issued % kStages;
                 const uint32_t ph = (k_issued / kStages) & 1;
-                if (!(ok = mbar_wait(&k_empty[s], ph ^ 1, abort_flag, &g_va_status))) break;
+                if (!(ok = mbar_wait_warp(&k_empty[s], ph ^ 1, abort_flag, &g_va_status))) break;
                 load_tile<D>(smem + L::kK + s * L::kTileBytes, &tmK, p.k, k0 + kt * kBlockN, T_k,
                              kv_stride, hk * D, &k_full[s], lane);
                 ++k_issued;
-                if (!(ok = mbar_wait(&v_empty[s], ph ^ 1, abort_flag, &g_va_status))) break;
+                if (!(ok = mbar_wait_warp(&v_empty[s], ph ^ 1, abort_flag, &g_va_status))) break;
                 load_tile<D>(smem + L::kV + s * L::kTileBytes, &tmV, p.v, k0 + kt * kBlockN, T_k,
                              kv_stride, hk * D, &v_full[s], lane);
                 ++v_issued;
@@ -302,18 +302,26 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             float m_ref = -INFINITY, l = 0.f;
             for (int j = 0; j < n; ++j, ++tile_cnt) {
                 const uint32_t sb = tile_cnt & 1;
-                if (!(ok = mbar_wait(&s_full[sb], (tile_cnt >> 1) & 1, abort_flag, &g_va_status))) break;
+                if (!(ok = mbar_wait_warp(&s_full[sb], (tile_cnt >> 1) & 1, abort_flag, &g_va_status))) break;
                 __syncwarp();
                 tc_fence_after();
                 const uint32_t sbase = tmem + lane_addr + (sb ? kTmemS1 : kTmemS0);
                 float s[kBlockN];
-#pragma unroll
-                for (int c = 0; c < kBlockN / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(sbase + c * 32, r);
+                {
+                    // all four loads in flight before a single wait
+                    uint32_t r0[32], r1[32], r2[32], r3[32];
+                    tmem_ld32(sbase + 0, r0);
+                    tmem_ld32(sbase + 32, r1);
+                    tmem_ld32(sbase + 64, r2);
+                    tmem_ld32(sbase + 96, r3);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(r[x]);
+                    for (int x = 0; x < 32; ++x) {
+                        s[x] = __uint_as_float(r0[x]);
+                        s[32 + x] = __uint_as_float(r1[x]);
+                        s[64 + x] = __uint_as_float(r2[x]);
+                        s[96 + x] = __uint_as_float(r3[x]);
+                    }
                 }
                 const int key0 = (te.kt_lo + j) * kBlockN;
                 const bool full_tile = lo <= key0 && key0 + kBlockN - 1 <= hi;
@@ -324,9 +332,16 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         s[c] = (kj >= lo && kj <= hi) ? s[c] : -INFINITY;
                     }
                 }
-                float mx = s[0];
+                // row max as a tree (short dependency chains)
+                float mv[8];
 #pragma unroll
-                for (int c = 1; c < kBlockN; ++c) mx = fmaxf(mx, s[c]);
+                for (int x = 0; x < 8; ++x) mv[x] = s[x];
+#pragma unroll
+                for (int c = 8; c < kBlockN; c += 8)
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) mv[x] = fmaxf(mv[x], s[c + x]);
+                const float mx = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
+                                       fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
                 const float m_tile = mx * p.scale_log2;  // -inf stays -inf
                 const float m_cand = fmaxf(m_ref, m_tile);
                 const bool want = (j == 0) || (m_cand > m_ref + kRescaleThreshold);
@@ -337,33 +352,39 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     m_ref = m_cand;
                 }
                 const float m_sub = (m_ref == -INFINITY) ? 0.f : m_ref;
-                float rowsum = 0.f;
+                float sums[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                 uint32_t pk[kBlockN / 2];
 #pragma unroll
                 for (int c = 0; c < kBlockN; c += 2) {
                     const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_sub));
                     const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_sub));
-                    rowsum += p0 + p1;
+                    sums[(c >> 1) & 7] += p0 + p1;
                     pk[c / 2] = pack_bf16x2(p0, p1);
                 }
+                const float rowsum = ((sums[0] + sums[1]) + (sums[2] + sums[3])) +
+                                     ((sums[4] + sums[5]) + (sums[6] + sums[7]));
                 l = l * alpha + rowsum;
                 if (j > 0) {
                     // O must hold P_{j-1} V_{j-1} before it is rescaled
-                    if (!(ok = mbar_wait(o_done, o_cnt & 1, abort_flag, &g_va_status))) break;
+                    if (!(ok = mbar_wait_warp(o_done, o_cnt & 1, abort_flag, &g_va_status))) break;
                     ++o_cnt;
                     __syncwarp();
                     tc_fence_after();
                     if (move) {
                         const uint32_t obase = tmem + lane_addr + kTmemO;
 #pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t r[32];
+                        for (int c = 0; c < D / 32; c += 2) {
+                            uint32_t r[32], r2[32];
                             tmem_ld32(obase + c * 32, r);
+                            tmem_ld32(obase + (c + 1) * 32, r2);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int x = 0; x < 32; ++x)
+                            for (int x = 0; x < 32; ++x) {
                                 r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
+                                r2[x] = __float_as_uint(__uint_as_float(r2[x]) * alpha);
+                            }
                             tmem_st32(obase + c * 32, r);
+                            tmem_st32(obase + (c + 1) * 32, r2);
                         }
                     }
                 }
@@ -384,7 +405,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             }
             if (!ok) break;
             // epilogue: wait for the last P V, then O / l and logsumexp
-            if (!(ok = mbar_wait(o_done, o_cnt & 1, abort_flag, &g_va_status))) break;
+            if (!(ok = mbar_wait_warp(o_done, o_cnt & 1, abort_flag, &g_va_status))) break;
             ++o_cnt;
             __syncwarp();
             tc_fence_after();

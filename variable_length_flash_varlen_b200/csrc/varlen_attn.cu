@@ -45,6 +45,10 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
     bool ready = false;
     int num_sms = 0;
+    // Library-private stream-ordered pool.  Its release threshold is
+    // unlimited, so a synchronisation does not hand its memory back to the OS
+    // and the next call does not pay for mapping it again.
+    cudaMemPool_t pool = nullptr;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -79,8 +83,25 @@ int device_setup(int& dev, DeviceInfo*& info) {
     VA_CUDA(cudaFuncSetAttribute(va::build_schedule_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  va::kSortCapacity * 8));
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    VA_CUDA(cudaMemPoolCreate(&info->pool, &props));
+    unsigned long long threshold = ~0ull;
+    VA_CUDA(cudaMemPoolSetAttribute(info->pool, cudaMemPoolAttrReleaseThreshold, &threshold));
     info->ready = true;
     return VA_OK;
+}
+
+// Stream-ordered workspace from the library pool of the current device.
+cudaError_t ws_alloc(void** p, size_t bytes, cudaStream_t stream) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices || !g_dev[dev].pool) return cudaErrorInitializationError;
+    return cudaMallocFromPoolAsync(p, bytes, g_dev[dev].pool, stream);
 }
 
 // 2-D bf16 view [rows][cols] (cols contiguous), box 64 x 128, 128-byte swizzle.
@@ -145,7 +166,7 @@ int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
     const size_t hdr_bytes = 256;
     const size_t list_bytes = static_cast<size_t>(cap) * sizeof(va::TileEntry);
     char* ws = nullptr;
-    VA_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&ws), hdr_bytes + 2 * list_bytes, stream));
+    VA_CUDA(ws_alloc(reinterpret_cast<void**>(&ws), hdr_bytes + 2 * list_bytes, stream));
     auto* hdr = reinterpret_cast<va::SchedHeader*>(ws);
     auto* scratch = reinterpret_cast<va::TileEntry*>(ws + hdr_bytes);
     auto* tiles = reinterpret_cast<va::TileEntry*>(ws + hdr_bytes + list_bytes);
@@ -212,7 +233,7 @@ int run_decode(const Args& a, int split_keys, cudaStream_t stream) {
     const size_t slots = static_cast<size_t>(a.batch) * a.H * n_split_max;
     char* ws = nullptr;
     const size_t o_bytes = slots * a.D * sizeof(float);
-    VA_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&ws), o_bytes + slots * 2 * sizeof(float), stream));
+    VA_CUDA(ws_alloc(reinterpret_cast<void**>(&ws), o_bytes + slots * 2 * sizeof(float), stream));
 
     va::DecodeParams p;
     p.cu_q = a.cu_q;
@@ -300,6 +321,9 @@ int varlen_attention_fwd_host(const void* q, const void* k, const void* v,
     if (rc != VA_OK) return rc;
     if (batch == 0 || max_seqlen_q == 0) return VA_OK;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    int dev;
+    DeviceInfo* info;
+    if ((rc = device_setup(dev, info)) != VA_OK) return rc;
     const long long T_q = cu_seqlens_q[batch], T_k = cu_seqlens_k[batch];
     if (T_q < 0 || T_k < 0) return fail(VA_ERR_INVALID_ARG, "negative total length");
     const size_t qb = static_cast<size_t>(T_q) * num_heads * head_dim * 2;
@@ -309,7 +333,7 @@ int varlen_attention_fwd_host(const void* q, const void* k, const void* v,
     auto up16 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
     const size_t total = up16(qb) + 2 * up16(kb) + 2 * up16(cb) + up16(ob) + up16(lb);
     char* ws = nullptr;
-    VA_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&ws), total, stream));
+    VA_CUDA(ws_alloc(reinterpret_cast<void**>(&ws), total, stream));
     char* p = ws;
     void* dq = p; p += up16(qb);
     void* dk = p; p += up16(kb);
@@ -361,7 +385,7 @@ int varlen_attention_schedule(const int32_t* cu_seqlens_q, const int32_t* cu_seq
     while (key_slots < capacity && key_slots < va::kSortCapacity) key_slots <<= 1;
     char* ws = nullptr;
     const size_t list_bytes = static_cast<size_t>(capacity) * sizeof(va::TileEntry);
-    VA_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&ws), 256 + list_bytes, stream));
+    VA_CUDA(ws_alloc(reinterpret_cast<void**>(&ws), 256 + list_bytes, stream));
     auto* hdr = reinterpret_cast<va::SchedHeader*>(ws);
     va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
         cu_seqlens_q, cu_seqlens_k, batch, causal ? 1 : 0, window, capacity, key_slots,
