@@ -107,14 +107,15 @@ int varlen_attention_fwd_host(const void* q, const void* k, const void* v,
                               int causal, int window, void* out, float* lse, void* stream);
 
 /*
- * The longest-first query-tile work list the prefill path builds from
- * cu_seqlens (device pointers), written to `tiles` (device int32
- * [capacity][4] = {sequence, query tile, first key tile, end key tile}) and
- * its length to `n_tiles` (device int32).  Tiles hold 128 query rows and 128
- * keys; key tiles [first, end) hold every key any row of the tile can see,
- * end == first when none.  Order: descending end - first, ties by ascending
- * (sequence, query tile).  capacity must be >= the number of query tiles,
- * otherwise *n_tiles = 0 and VA_STATUS_SCHEDULE_OVERFLOW is raised.
+ * The longest-first work list the prefill path builds from cu_seqlens
+ * (device pointers), written to `tiles` (device int32 [capacity][4] =
+ * {sequence, query block, first key tile, end key tile}) and its length to
+ * `n_tiles` (device int32).  A query block holds 256 query rows, a key tile
+ * 128 keys; key tiles [first, end) hold every key any row of the block can
+ * see, end == first when none.  Order: descending end - first, ties by
+ * ascending (sequence, query block).  capacity must be >= the number of
+ * query blocks, otherwise *n_tiles = 0 and VA_STATUS_SCHEDULE_OVERFLOW is
+ * raised.
  */
 int varlen_attention_schedule(const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
                               int batch, int max_seqlen_q, int causal, int window,

@@ -1,12 +1,12 @@
 """CPU statement of the tile work list (test infrastructure only).
 
-The GPU path splits every sequence's queries into tiles of ``BLOCK_M`` rows and
-walks keys in tiles of ``BLOCK_N``.  For each query tile it needs the
-half-open range of key tiles [kt_lo, kt_hi) that holds every key visible to
-any row of the tile; the tiles outside it are skipped (boostr flash.rs,
+The GPU path splits every sequence's queries into blocks of ``BLOCK_M`` rows
+(one work item each) and walks keys in tiles of ``BLOCK_N``.  For each query
+block it needs the half-open range of key tiles [kt_lo, kt_hi) that holds
+every key visible to any row of the block; the tiles outside it are skipped (boostr flash.rs,
 FlashAttentionOps docs, "Sliding window": whole K/V tiles outside the window
 are skipped).  The list is ordered longest first: by descending tile count,
-ties by ascending (sequence, query tile).  This module computes that list
+ties by ascending (sequence, query block).  This module computes that list
 from host cu_seqlens with plain Python so that the device-built list can be
 compared with it entry by entry.
 
@@ -18,7 +18,7 @@ from __future__ import annotations
 
 from typing import List, Sequence, Tuple
 
-BLOCK_M = 128
+BLOCK_M = 256
 BLOCK_N = 128
 
 

@@ -157,7 +157,7 @@ def test_schedule_bit_exact(name, scale):
     wl = workloads.named(name, scale=scale)
     cq = torch.tensor(wl.cu_q, dtype=torch.int32, device="cuda")
     ck = torch.tensor(wl.cu_k, dtype=torch.int32, device="cuda")
-    cap = wl.batch * ((wl.max_seqlen_q + 127) // 128)
+    cap = wl.batch * ((wl.max_seqlen_q + 255) // 256)
     got = binding.varlen_attention_schedule(cq, ck, wl.batch, wl.max_seqlen_q, wl.causal,
                                             wl.window, cap).cpu().numpy()
     want = np.array(sch.schedule(wl.cu_q, wl.cu_k, wl.causal, wl.window), dtype=np.int32)
@@ -171,7 +171,7 @@ def test_schedule_edge_lists_bit_exact():
                               ([1000, 300], [1000, 300], False, 200)]:
         cq = torch.tensor(workloads.cu_seqlens(Lq), dtype=torch.int32, device="cuda")
         ck = torch.tensor(workloads.cu_seqlens(Lk), dtype=torch.int32, device="cuda")
-        cap = len(Lq) * ((max(Lq) + 127) // 128)
+        cap = len(Lq) * ((max(Lq) + 255) // 256)
         got = binding.varlen_attention_schedule(cq, ck, len(Lq), max(Lq), causal, W, cap)
         want = sch.schedule(workloads.cu_seqlens(Lq), workloads.cu_seqlens(Lk), causal, W)
         assert [tuple(r) for r in got.cpu().tolist()] == want

@@ -1,24 +1,31 @@
 // Persistent, warp-specialised packed-attention forward for sm_100a.
 //
-// Per CTA (192 threads, one CTA per SM):
-//   warp 0      producer: TMA tile loads of Q, K, V into 128-byte-swizzled
+// A work item is one 256-row query block of one (sequence, query head),
+// split into two 128-row MMA tiles ("halves") that share every K/V tile of
+// 128 keys.  Per CTA (320 threads, one CTA per SM):
+//   warps 0-3   softmax for half 0, warps 4-7 softmax for half 1: one query
+//               row per thread; online softmax in base 2 with a lazily moved
+//               reference max, P written back to tensor memory as bf16, O
+//               rescaled in place when the reference moves, epilogue O / l
+//               and logsumexp
+//   warp 8      tensor-memory owner and MMA issuer (one lane):
+//               S_h = Q_h K^T (SS form), O_h += P_h V (P_h read from tensor
+//               memory), issued as PV_0[j], QK_0[j+1], PV_1[j], QK_1[j+1] so
+//               one half's MMAs run while the other half's softmax does
+//   warp 9      producer: claims work items from a grid-wide counter (longest
+//               first), TMA tile loads of Q, K, V into 128-byte-swizzled
 //               shared memory (plain loads for a tile that runs past the end
 //               of the packed tensor)
-//   warp 1      tensor-memory owner and MMA issuer: one lane issues
-//               S = Q K^T (SS form) and O += P V (P read from tensor memory)
-//   warps 2-5   softmax: one query row per thread; online softmax in base 2
-//               with a lazily moved reference max, P written back to tensor
-//               memory as bf16, O rescaled in place, epilogue O / l and
-//               logsumexp
-// Tensor memory (512 columns): S/P double buffer at columns 0 and 128, O at 256.
+// Tensor memory (512 columns): S_0 at 0, S_1 at 128 (P_h aliases the first
+// 64 columns of S_h), O_0 at 256, O_1 at 256 + D.
 //
 // The recurrence is the tiled one of realizar 0.8.4 attention.rs, IMP-111
 // (online_softmax / tiled_single_head_attention): running max, running sum
 // rescaled by exp(old - new), output rescaled alongside, normalised at the end.
 // Packed addressing and GQA head mapping follow boostr 0.2.0
 // varlen_attention.rs, VarLenAttentionOps docs ("Layout contract", "GQA
-// key/value head mapping"): kv_head = q_head / (H / H_kv), K/V read once per
-// tile for the head that needs them, never repeated in memory.
+// key/value head mapping"): kv_head = q_head / (H / H_kv); K/V are read for
+// the head that needs them and never repeated in memory.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -29,10 +36,11 @@
 
 namespace va {
 
-constexpr int kPrefillThreads = 192;
-constexpr int kStages = 2;             // K/V ring depth
+constexpr int kPrefillThreads = 320;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr int kStages = 2;  // K/V ring depth (tiles of kBlockN keys)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow to 2^8 before O is rescaled
 
 struct PrefillParams {
@@ -40,7 +48,7 @@ struct PrefillParams {
     const int* cu_k;
     int batch, H, H_kv, causal, window;
     const TileEntry* tiles;
-    const SchedHeader* hdr;
+    SchedHeader* hdr;
     int tile_capacity;  // entries the list can hold; the count read from hdr is clamped to it
     const __nv_bfloat16* q;
     const __nv_bfloat16* k;
@@ -52,21 +60,56 @@ struct PrefillParams {
 
 template <int D>
 struct PrefillSmem {
-    static constexpr int kChunks = D / 64;                 // 128-byte swizzle atoms per row
-    static constexpr int kChunkBytes = 128 * 128;          // 128 rows x 128 bytes
+    static constexpr int kChunks = D / 64;          // 128-byte swizzle atoms per row
+    static constexpr int kChunkBytes = 128 * 128;   // 128 rows x 128 bytes
     static constexpr int kTileBytes = kChunks * kChunkBytes;
-    static constexpr int kQ = 0;
-    static constexpr int kK = kQ + kTileBytes;
+    static constexpr int kQ = 0;                    // two Q tiles
+    static constexpr int kK = kQ + 2 * kTileBytes;
     static constexpr int kV = kK + kStages * kTileBytes;
     static constexpr int kBar = kV + kStages * kTileBytes;
-    // barriers: q_full, q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_done
-    static constexpr int kNumBars = 2 + 4 * kStages + 5;
+    // q_full[2], q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
+    // o_done[2], item_full[2], item_empty[2]
+    static constexpr int kNumBars = 3 + 4 * kStages + 10;
     static constexpr int kMisc = kBar + kNumBars * 8;
-    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kBytes = kMisc + 16;  // tmem slot, abort flag, item ring[2]
     // slack for 1024-byte alignment; never below 120 KB so that at most one CTA
     // (and one 512-column tensor-memory allocation) is resident per SM
     static constexpr int kAlloc = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
+    __host__ __device__ static constexpr uint32_t tmem_s(int x) { return x ? 128u : 0u; }
+    __host__ __device__ static constexpr uint32_t tmem_o(int x) { return 256u + x * D; }
 };
+
+// Everything every role derives from a work-item index.
+struct Item {
+    int b, qb, h, hk;
+    int L_q, L_k;
+    int q_row0, k_row0;   // first packed row of the query block / of the sequence's keys
+    int lo, hi;           // key-tile range of the block (union of the halves)
+    int lo_h[2], hi_h[2]; // key-tile range of each 128-row half
+};
+
+__device__ __forceinline__ void decode_item(const PrefillParams& p, int idx, int group, Item& it) {
+    const TileEntry te = p.tiles[idx / p.H];
+    it.h = idx % p.H;
+    it.hk = it.h / group;
+    it.b = te.b;
+    it.qb = te.qt;
+    it.lo = te.kt_lo;
+    it.hi = te.kt_hi;
+    const int cq = p.cu_q[it.b], ck = p.cu_k[it.b];
+    it.L_q = p.cu_q[it.b + 1] - cq;
+    it.L_k = p.cu_k[it.b + 1] - ck;
+    it.q_row0 = cq + it.qb * kBlockQ;
+    it.k_row0 = ck;
+#pragma unroll
+    for (int x = 0; x < 2; ++x)
+        rows_key_range(it.qb * kBlockQ + x * kBlockM, kBlockM, it.L_q, it.L_k, p.causal != 0,
+                       p.window, it.lo_h[x], it.hi_h[x]);
+}
+
+__device__ __forceinline__ bool takes_part(const Item& it, int x, int kt) {
+    return it.lo_h[x] <= kt && kt < it.hi_h[x];
+}
 
 // Copy a 128-row tile whose rows may run past `T` with plain loads, writing
 // the 128-byte-swizzle layout TMA would have produced; rows >= T become zero.
@@ -89,6 +132,7 @@ __device__ __forceinline__ void load_tile_plain(uint8_t* dst, const __nv_bfloat1
     __syncwarp();
 }
 
+// Whole warp: one 128-row tile into `dst`, completion signalled on `full`.
 template <int D>
 __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map,
                                           const __nv_bfloat16* src, int row0, int T, int row_stride,
@@ -109,6 +153,14 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map,
 }
 
 template <int D>
+__device__ __forceinline__ void store_row_zero(const PrefillParams& p, size_t out_row) {
+    uint4* o4 = reinterpret_cast<uint4*>(p.out + out_row * D);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) o4[c] = make_uint4(0u, 0u, 0u, 0u);
+    p.lse[out_row] = -INFINITY;
+}
+
+template <int D>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
@@ -117,22 +169,32 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-    uint64_t* q_full = bars + 0;
-    uint64_t* q_empty = bars + 1;
-    uint64_t* k_full = bars + 2;
+    uint64_t* q_full = bars + 0;  // [2]
+    uint64_t* q_empty = bars + 2;
+    uint64_t* k_full = bars + 3;
     uint64_t* k_empty = k_full + kStages;
     uint64_t* v_full = k_empty + kStages;
     uint64_t* v_empty = v_full + kStages;
-    uint64_t* s_full = v_empty + kStages;
-    uint64_t* p_full = s_full + 2;
-    uint64_t* o_done = p_full + 2;
+    uint64_t* s_full = v_empty + kStages;  // [2]
+    uint64_t* p_full = s_full + 2;         // [2]
+    uint64_t* o_done = p_full + 2;         // [2]
+    uint64_t* item_full = o_done + 2;      // [2]
+    uint64_t* item_empty = item_full + 2;  // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+    volatile int* item_ring = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [2]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&q_full[x], 1);
+            mbar_init(&s_full[x], 1);
+            mbar_init(&p_full[x], 4);
+            mbar_init(&o_done[x], 1);
+            mbar_init(&item_full[x], 1);
+            mbar_init(&item_empty[x], 1 + 8);  // the MMA lane and the eight softmax warps
+        }
         mbar_init(q_empty, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&k_full[s], 1);
@@ -140,19 +202,14 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&s_full[s], 1);
-            mbar_init(&p_full[s], 4);
-        }
-        mbar_init(o_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == kLoadWarp && lane == 0) {
         prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
@@ -164,32 +221,54 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
     const int n_items = min(max(p.hdr->n_tiles, 0), p.tile_capacity) * p.H;
     const int group = p.H / p.H_kv;
+    unsigned* status = &g_va_status;
 
-    if (warp == 0) {
+    if (warp == kLoadWarp) {
         // ------------------------------------------------------------ producer
         const int T_q = p.cu_q[p.batch], T_k = p.cu_k[p.batch];
         const int q_stride = p.H * D, kv_stride = p.H_kv * D;
-        uint32_t q_issued = 0, k_issued = 0, v_issued = 0;
+        uint32_t items_done = 0, q_issued[2] = {0, 0}, k_issued = 0, v_issued = 0, ring = 0;
         bool ok = true;
-        for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
-            const TileEntry te = p.tiles[idx / p.H];
-            const int h = idx % p.H, hk = h / group;
-            if (te.kt_hi <= te.kt_lo) continue;
-            if (!(ok = mbar_wait_warp(q_empty, (q_issued & 1) ^ 1, abort_flag, &g_va_status))) break;
-            load_tile<D>(smem + L::kQ, &tmQ, p.q, p.cu_q[te.b] + te.qt * kBlockM, T_q, q_stride,
-                         h * D, q_full, lane);
-            ++q_issued;
-            const int k0 = p.cu_k[te.b];
-            for (int kt = te.kt_lo; kt < te.kt_hi; ++kt) {
+        for (;;) {
+            // claim the next work item (longest first across the grid) and publish it
+            int idx = -1;
+            if (lane == 0) {
+                const int t = atomicAdd(&p.hdr->next_item, 1);
+                idx = t < n_items ? t : -1;
+            }
+            idx = __shfl_sync(0xffffffffu, idx, 0);
+            if (!(ok = mbar_wait_warp(&item_empty[ring & 1], ((ring >> 1) & 1) ^ 1, abort_flag, status)))
+                break;
+            if (lane == 0) {
+                item_ring[ring & 1] = idx;
+                mbar_arrive(&item_full[ring & 1]);
+            }
+            __syncwarp();
+            ++ring;
+            if (idx < 0) break;
+            Item it;
+            decode_item(p, idx, group, it);
+            if (it.hi <= it.lo) continue;
+            if (!(ok = mbar_wait_warp(q_empty, (items_done & 1) ^ 1, abort_flag, status))) break;
+            ++items_done;
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                if (it.hi_h[x] > it.lo_h[x]) {
+                    load_tile<D>(smem + L::kQ + x * L::kTileBytes, &tmQ, p.q, it.q_row0 + x * kBlockM,
+                                 T_q, q_stride, it.h * D, &q_full[x], lane);
+                    ++q_issued[x];
+                }
+            }
+            for (int kt = it.lo; kt < it.hi; ++kt) {
                 const int s = k_issued % kStages;
                 const uint32_t ph = (k_issued / kStages) & 1;
-                if (!(ok = mbar_wait_warp(&k_empty[s], ph ^ 1, abort_flag, &g_va_status))) break;
-                load_tile<D>(smem + L::kK + s * L::kTileBytes, &tmK, p.k, k0 + kt * kBlockN, T_k,
-                             kv_stride, hk * D, &k_full[s], lane);
+                if (!(ok = mbar_wait_warp(&k_empty[s], ph ^ 1, abort_flag, status))) break;
+                load_tile<D>(smem + L::kK + s * L::kTileBytes, &tmK, p.k, it.k_row0 + kt * kBlockN,
+                             T_k, kv_stride, it.hk * D, &k_full[s], lane);
                 ++k_issued;
-                if (!(ok = mbar_wait_warp(&v_empty[s], ph ^ 1, abort_flag, &g_va_status))) break;
-                load_tile<D>(smem + L::kV + s * L::kTileBytes, &tmV, p.v, k0 + kt * kBlockN, T_k,
-                             kv_stride, hk * D, &v_full[s], lane);
+                if (!(ok = mbar_wait_warp(&v_empty[s], ph ^ 1, abort_flag, status))) break;
+                load_tile<D>(smem + L::kV + s * L::kTileBytes, &tmV, p.v, it.k_row0 + kt * kBlockN,
+                             T_k, kv_stride, it.hk * D, &v_full[s], lane);
                 ++v_issued;
             }
         }
@@ -203,109 +282,159 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                        global_timer_ns() - t0 < kWaitLimitNs) {
                 }
             };
-            drain(q_full, q_issued);
+            drain(&q_full[0], q_issued[0]);
+            drain(&q_full[1], q_issued[1]);
             for (int s = 0; s < kStages; ++s) {
-                // loads into stage s: indices s, s + kStages, ...
                 const uint32_t nk = k_issued > (uint32_t)s ? (k_issued - s + kStages - 1) / kStages : 0;
                 const uint32_t nv = v_issued > (uint32_t)s ? (v_issued - s + kStages - 1) / kStages : 0;
                 drain(&k_full[s], nk);
                 drain(&v_full[s], nv);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kBlockN, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-            const uint32_t sQ = smem_u32(smem + L::kQ);
-            const uint32_t sK = smem_u32(smem + L::kK);
-            const uint32_t sV = smem_u32(smem + L::kV);
-            uint32_t item_cnt = 0, kv_cnt = 0, tile_cnt = 0;
+            // descriptors: one high word per operand kind, low words stepped by the
+            // start-address field (16-byte units)
+            static_assert(L::kBar < (1 << 18), "descriptor start-address field covers 256 KB");
+            const uint64_t dq = smem_desc_sw128(smem_u32(smem + L::kQ), 16, 1024);
+            const uint64_t dk = smem_desc_sw128(smem_u32(smem + L::kK), 16, 1024);
+            const uint64_t dv = smem_desc_sw128(smem_u32(smem + L::kV), L::kChunkBytes, 1024);
+            const uint32_t q_lo = static_cast<uint32_t>(dq), q_hi = static_cast<uint32_t>(dq >> 32);
+            const uint32_t k_lo = static_cast<uint32_t>(dk), k_hi = static_cast<uint32_t>(dk >> 32);
+            const uint32_t v_lo = static_cast<uint32_t>(dv), v_hi = static_cast<uint32_t>(dv >> 32);
+            uint32_t q_waits[2] = {0, 0}, p_waits[2] = {0, 0}, kv = 0, ring = 0;
             bool ok = true;
-            // O += P V for the tile with global counters (kv index, tile index)
-            auto issue_pv = [&](uint32_t kv_i, uint32_t tile_i, bool first) -> bool {
-                const uint32_t sb = tile_i & 1;
-                if (!mbar_wait(&p_full[sb], (tile_i >> 1) & 1, abort_flag, &g_va_status)) return false;
-                const int s = kv_i % kStages;
-                if (!mbar_wait(&v_full[s], (kv_i / kStages) & 1, abort_flag, &g_va_status)) return false;
-                tc_fence_after();
-                const uint32_t vbase = sV + s * L::kTileBytes;
-                const uint32_t pbase = tmem + (sb ? kTmemS1 : kTmemS0);
+
+            auto issue_qk = [&](int x, int s) {
+                const uint32_t qa = q_lo + ((x * L::kTileBytes) >> 4);
+                const uint32_t kb = k_lo + ((s * L::kTileBytes) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4;
+                    mma_ss_lh<idesc_qk>(tmem + L::tmem_s(x), qa + off, q_hi, kb + off, k_hi,
+                                        kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&s_full[x]);
+            };
+            auto issue_pv = [&](int x, int s, bool first) {
+                const uint32_t vb = v_lo + ((s * L::kTileBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    const uint64_t bdesc = smem_desc_sw128(vbase + kk * 16 * 128, L::kChunkBytes, 1024);
-                    mma_ts(tmem + kTmemO, pbase + kk * 8, bdesc, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+                    mma_ts_lh<idesc_pv>(tmem + L::tmem_o(x), tmem + L::tmem_s(x) + kk * 8,
+                                        vb + ((kk * 16 * 128) >> 4), v_hi, (!first || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(o_done);
-                mma_commit(&v_empty[s]);
-                return true;
+                mma_commit(&o_done[x]);
             };
-            for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
-                const TileEntry te = p.tiles[idx / p.H];
-                const int n = te.kt_hi - te.kt_lo;
-                if (n <= 0) continue;
-                if (!(ok = mbar_wait(q_full, item_cnt & 1, abort_flag, &g_va_status))) break;
-                const uint32_t kv_base = kv_cnt, tile_base = tile_cnt;
-                for (int j = 0; j < n; ++j) {
-                    const uint32_t kv_i = kv_base + j, tile_i = tile_base + j;
-                    const int s = kv_i % kStages;
-                    if (!(ok = mbar_wait(&k_full[s], (kv_i / kStages) & 1, abort_flag, &g_va_status))) break;
-                    tc_fence_after();
-                    const uint32_t kbase = sK + s * L::kTileBytes;
-                    const uint32_t sdst = tmem + ((tile_i & 1) ? kTmemS1 : kTmemS0);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                        mma_ss(sdst, smem_desc_sw128(sQ + off, 16, 1024),
-                               smem_desc_sw128(kbase + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&s_full[tile_i & 1]);
-                    mma_commit(&k_empty[s]);
-                    if (j == n - 1) mma_commit(q_empty);
-                    if (j > 0 && !(ok = issue_pv(kv_i - 1, tile_i - 1, j - 1 == 0))) break;
+
+            for (;;) {
+                if (!(ok = mbar_wait(&item_full[ring & 1], (ring >> 1) & 1, abort_flag, status))) break;
+                const int idx = item_ring[ring & 1];
+                mbar_arrive(&item_empty[ring & 1]);
+                ++ring;
+                if (idx < 0) break;
+                Item it;
+                decode_item(p, idx, group, it);
+                if (it.hi <= it.lo) continue;
+                const int n = it.hi - it.lo;
+                for (int x = 0; x < 2 && ok; ++x) {
+                    if (it.hi_h[x] > it.lo_h[x])
+                        ok = mbar_wait(&q_full[x], q_waits[x]++ & 1, abort_flag, status);
                 }
                 if (!ok) break;
-                if (!(ok = issue_pv(kv_base + n - 1, tile_base + n - 1, n == 1))) break;
-                kv_cnt += n;
-                tile_cnt += n;
-                ++item_cnt;
+                // prologue: S for the first key tile
+                {
+                    const int s = kv % kStages;
+                    if (!(ok = mbar_wait(&k_full[s], (kv / kStages) & 1, abort_flag, status))) break;
+                    tc_fence_after();
+                    for (int x = 0; x < 2; ++x)
+                        if (takes_part(it, x, it.lo)) issue_qk(x, s);
+                    mma_commit(&k_empty[s]);
+                    if (n == 1) mma_commit(q_empty);  // last reader of Q issued
+                }
+                bool first_pv[2] = {true, true};
+                for (int j = 0; j < n && ok; ++j) {
+                    const int kt = it.lo + j;
+                    const uint32_t kv_j = kv + j, kv_n = kv + j + 1;
+                    const int s = kv_j % kStages, s_n = kv_n % kStages;
+                    const bool has_next = j + 1 < n;
+                    bool next_k_ready = false;
+                    if (!(ok = mbar_wait(&v_full[s], (kv_j / kStages) & 1, abort_flag, status))) break;
+                    for (int x = 0; x < 2 && ok; ++x) {
+                        if (takes_part(it, x, kt)) {
+                            if (!(ok = mbar_wait(&p_full[x], p_waits[x]++ & 1, abort_flag, status))) break;
+                            tc_fence_after();
+                            issue_pv(x, s, first_pv[x]);
+                            first_pv[x] = false;
+                        }
+                        if (has_next && takes_part(it, x, kt + 1)) {
+                            if (!next_k_ready) {
+                                if (!(ok = mbar_wait(&k_full[s_n], (kv_n / kStages) & 1, abort_flag, status)))
+                                    break;
+                                tc_fence_after();
+                                next_k_ready = true;
+                            }
+                            issue_qk(x, s_n);
+                        }
+                    }
+                    if (!ok) break;
+                    if (has_next) {
+                        if (!next_k_ready) {
+                            // every tile of the union has a taker; this wait only keeps
+                            // the ring's phases in step if that ever changes
+                            if (!(ok = mbar_wait(&k_full[s_n], (kv_n / kStages) & 1, abort_flag, status)))
+                                break;
+                        }
+                        mma_commit(&k_empty[s_n]);
+                        // the QKs of the last key tile are issued: Q may be reloaded as
+                        // soon as they complete, while the last softmax and PV run
+                        if (j + 2 == n) mma_commit(q_empty);
+                    }
+                    mma_commit(&v_empty[s]);
+                }
+                if (!ok) break;
+                kv += n;
             }
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax
-        const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
-        const int row = quarter * 32 + lane;          // query row within the tile
+        const int x = warp >> 2;                    // which half of the query block
+        const int quarter = warp & 3;               // TMEM lane quarter this warp may access
+        const int row_in_tile = quarter * 32 + lane;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-        uint32_t tile_cnt = 0, o_cnt = 0;
+        const uint32_t sbase = tmem + lane_addr + L::tmem_s(x);
+        const uint32_t obase = tmem + lane_addr + L::tmem_o(x);
+        uint32_t s_waits = 0, o_waits = 0, ring = 0;
         bool ok = true;
-        for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x) {
-            const TileEntry te = p.tiles[idx / p.H];
-            const int h = idx % p.H;
-            const int L_q = p.cu_q[te.b + 1] - p.cu_q[te.b];
-            const int L_k = p.cu_k[te.b + 1] - p.cu_k[te.b];
-            const int i = te.qt * kBlockM + row;
-            const bool row_valid = i < L_q;
+        for (;;) {
+            if (!(ok = mbar_wait_warp(&item_full[ring & 1], (ring >> 1) & 1, abort_flag, status))) break;
+            const int idx = item_ring[ring & 1];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&item_empty[ring & 1]);
+            ++ring;
+            if (idx < 0) break;
+            Item it;
+            decode_item(p, idx, group, it);
+            const int i = it.qb * kBlockQ + x * kBlockM + row_in_tile;
+            const bool row_valid = i < it.L_q;
             int lo, hi;
-            row_key_interval(i, L_q, L_k, p.causal != 0, p.window, lo, hi);
-            const size_t out_row = static_cast<size_t>(p.cu_q[te.b] + i) * p.H + h;
-            const int n = te.kt_hi - te.kt_lo;
-            if (n <= 0) {
-                if (row_valid) {
-                    uint4* o4 = reinterpret_cast<uint4*>(p.out + out_row * D);
-#pragma unroll
-                    for (int c = 0; c < D / 8; ++c) o4[c] = make_uint4(0u, 0u, 0u, 0u);
-                    p.lse[out_row] = -INFINITY;
-                }
+            row_key_interval(i, it.L_q, it.L_k, p.causal != 0, p.window, lo, hi);
+            const size_t out_row = static_cast<size_t>(it.q_row0 + x * kBlockM + row_in_tile) * p.H + it.h;
+            if (it.hi_h[x] <= it.lo_h[x]) {
+                if (row_valid) store_row_zero<D>(p, out_row);
                 continue;
             }
+            // keys every row of this warp sees: tiles inside [warp_lo, warp_hi] need no mask
+            const int warp_lo = __reduce_max_sync(0xffffffffu, lo);
+            const int warp_hi = __reduce_min_sync(0xffffffffu, hi);
             float m_ref = -INFINITY, l = 0.f;
-            for (int j = 0; j < n; ++j, ++tile_cnt) {
-                const uint32_t sb = tile_cnt & 1;
-                if (!(ok = mbar_wait_warp(&s_full[sb], (tile_cnt >> 1) & 1, abort_flag, &g_va_status))) break;
-                __syncwarp();
+            for (int kt = it.lo_h[x]; kt < it.hi_h[x]; ++kt) {
+                const bool first_tile = kt == it.lo_h[x];
+                if (!(ok = mbar_wait_warp(&s_full[x], s_waits++ & 1, abort_flag, status))) break;
                 tc_fence_after();
-                const uint32_t sbase = tmem + lane_addr + (sb ? kTmemS1 : kTmemS0);
                 float s[kBlockN];
                 {
                     // all four loads in flight before a single wait
@@ -316,16 +445,15 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     tmem_ld32(sbase + 96, r3);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) {
-                        s[x] = __uint_as_float(r0[x]);
-                        s[32 + x] = __uint_as_float(r1[x]);
-                        s[64 + x] = __uint_as_float(r2[x]);
-                        s[96 + x] = __uint_as_float(r3[x]);
+                    for (int c = 0; c < 32; ++c) {
+                        s[c] = __uint_as_float(r0[c]);
+                        s[32 + c] = __uint_as_float(r1[c]);
+                        s[64 + c] = __uint_as_float(r2[c]);
+                        s[96 + c] = __uint_as_float(r3[c]);
                     }
                 }
-                const int key0 = (te.kt_lo + j) * kBlockN;
-                const bool full_tile = lo <= key0 && key0 + kBlockN - 1 <= hi;
-                if (__any_sync(0xffffffffu, !full_tile)) {
+                const int key0 = kt * kBlockN;
+                if (!(warp_lo <= key0 && key0 + kBlockN - 1 <= warp_hi)) {
 #pragma unroll
                     for (int c = 0; c < kBlockN; ++c) {
                         const int kj = key0 + c;
@@ -335,16 +463,16 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 // row max as a tree (short dependency chains)
                 float mv[8];
 #pragma unroll
-                for (int x = 0; x < 8; ++x) mv[x] = s[x];
+                for (int c = 0; c < 8; ++c) mv[c] = s[c];
 #pragma unroll
                 for (int c = 8; c < kBlockN; c += 8)
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) mv[x] = fmaxf(mv[x], s[c + x]);
+                    for (int e = 0; e < 8; ++e) mv[e] = fmaxf(mv[e], s[c + e]);
                 const float mx = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
                                        fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
                 const float m_tile = mx * p.scale_log2;  // -inf stays -inf
                 const float m_cand = fmaxf(m_ref, m_tile);
-                const bool want = (j == 0) || (m_cand > m_ref + kRescaleThreshold);
+                const bool want = first_tile || (m_cand > m_ref + kRescaleThreshold);
                 const bool move = __any_sync(0xffffffffu, want);
                 float alpha = 1.f;
                 if (move) {
@@ -352,65 +480,50 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     m_ref = m_cand;
                 }
                 const float m_sub = (m_ref == -INFINITY) ? 0.f : m_ref;
+                // P = 2^(s * scale_log2 - m_ref) as bf16 pairs into S_x, 32 columns at a
+                // time.  S_x's previous P was consumed by the PV issued before this QK.
                 float sums[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                uint32_t pk[kBlockN / 2];
 #pragma unroll
-                for (int c = 0; c < kBlockN; c += 2) {
-                    const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_sub));
-                    const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_sub));
-                    sums[(c >> 1) & 7] += p0 + p1;
-                    pk[c / 2] = pack_bf16x2(p0, p1);
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 64; c += 2) {
+                        const float p0 = ex2_approx(fmaf(s[half * 64 + c], p.scale_log2, -m_sub));
+                        const float p1 = ex2_approx(fmaf(s[half * 64 + c + 1], p.scale_log2, -m_sub));
+                        sums[(c >> 1) & 7] += p0 + p1;
+                        pk[c / 2] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st32(sbase + half * 32, pk);
                 }
-                const float rowsum = ((sums[0] + sums[1]) + (sums[2] + sums[3])) +
-                                     ((sums[4] + sums[5]) + (sums[6] + sums[7]));
-                l = l * alpha + rowsum;
-                if (j > 0) {
-                    // O must hold P_{j-1} V_{j-1} before it is rescaled
-                    if (!(ok = mbar_wait_warp(o_done, o_cnt & 1, abort_flag, &g_va_status))) break;
-                    ++o_cnt;
-                    __syncwarp();
+                l = l * alpha + (((sums[0] + sums[1]) + (sums[2] + sums[3])) +
+                                 ((sums[4] + sums[5]) + (sums[6] + sums[7])));
+                if (!first_tile) {
+                    // O_x must hold every earlier P V before it is rescaled
+                    if (!(ok = mbar_wait_warp(&o_done[x], o_waits++ & 1, abort_flag, status))) break;
                     tc_fence_after();
                     if (move) {
-                        const uint32_t obase = tmem + lane_addr + kTmemO;
 #pragma unroll
-                        for (int c = 0; c < D / 32; c += 2) {
-                            uint32_t r[32], r2[32];
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t r[32];
                             tmem_ld32(obase + c * 32, r);
-                            tmem_ld32(obase + (c + 1) * 32, r2);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int x = 0; x < 32; ++x) {
-                                r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
-                                r2[x] = __float_as_uint(__uint_as_float(r2[x]) * alpha);
-                            }
+                            for (int e = 0; e < 32; ++e)
+                                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
                             tmem_st32(obase + c * 32, r);
-                            tmem_st32(obase + (c + 1) * 32, r2);
                         }
                     }
-                }
-                {
-                    uint32_t r0[32], r1[32];
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) {
-                        r0[x] = pk[x];
-                        r1[x] = pk[32 + x];
-                    }
-                    tmem_st32(sbase, r0);
-                    tmem_st32(sbase + 32, r1);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[sb]);
+                if (lane == 0) mbar_arrive(&p_full[x]);
             }
             if (!ok) break;
             // epilogue: wait for the last P V, then O / l and logsumexp
-            if (!(ok = mbar_wait_warp(o_done, o_cnt & 1, abort_flag, &g_va_status))) break;
-            ++o_cnt;
-            __syncwarp();
+            if (!(ok = mbar_wait_warp(&o_done[x], o_waits++ & 1, abort_flag, status))) break;
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            const uint32_t obase = tmem + lane_addr + kTmemO;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t r[32];
@@ -419,13 +532,13 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 if (row_valid) {
                     uint4* o4 = reinterpret_cast<uint4*>(p.out + out_row * D + c * 32);
 #pragma unroll
-                    for (int x = 0; x < 4; ++x) {
+                    for (int e = 0; e < 4; ++e) {
                         uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(r[8 * x + 0]) * inv_l, __uint_as_float(r[8 * x + 1]) * inv_l);
-                        w.y = pack_bf16x2(__uint_as_float(r[8 * x + 2]) * inv_l, __uint_as_float(r[8 * x + 3]) * inv_l);
-                        w.z = pack_bf16x2(__uint_as_float(r[8 * x + 4]) * inv_l, __uint_as_float(r[8 * x + 5]) * inv_l);
-                        w.w = pack_bf16x2(__uint_as_float(r[8 * x + 6]) * inv_l, __uint_as_float(r[8 * x + 7]) * inv_l);
-                        o4[x] = w;
+                        w.x = pack_bf16x2(__uint_as_float(r[8 * e + 0]) * inv_l, __uint_as_float(r[8 * e + 1]) * inv_l);
+                        w.y = pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv_l, __uint_as_float(r[8 * e + 3]) * inv_l);
+                        w.z = pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv_l, __uint_as_float(r[8 * e + 5]) * inv_l);
+                        w.w = pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv_l, __uint_as_float(r[8 * e + 7]) * inv_l);
+                        o4[e] = w;
                     }
                 }
             }
@@ -438,7 +551,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);

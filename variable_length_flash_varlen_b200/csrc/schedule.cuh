@@ -1,7 +1,8 @@
 // Work list of query tiles, built on the device from cu_seqlens.
 //
-// Every sequence b's queries are cut into tiles of kBlockM rows; for each
-// tile the key tiles (kBlockN keys) that any of its rows can see form the
+// Every sequence b's queries are cut into blocks of kBlockQ rows (one work
+// item; the kernel splits it into two MMA tiles of kBlockM rows); for each
+// block the key tiles (kBlockN keys) that any of its rows can see form the
 // half-open range [kt_lo, kt_hi).  Key tiles outside the range are never
 // loaded: the causal triangle above the diagonal and the keys older than a
 // sliding window (boostr flash.rs, FlashAttentionOps docs, "Sliding window")
@@ -16,12 +17,13 @@
 
 namespace va {
 
-constexpr int kBlockM = 128;   // query rows per tile
+constexpr int kBlockM = 128;   // query rows per MMA tile
+constexpr int kBlockQ = 256;   // query rows per work item (two MMA tiles)
 constexpr int kBlockN = 128;   // keys per tile
-constexpr int kSortCapacity = 16384;  // query tiles sorted in shared memory
+constexpr int kSortCapacity = 16384;  // query blocks sorted in shared memory
 
 struct TileEntry {
-    int b, qt, kt_lo, kt_hi;
+    int b, qt, kt_lo, kt_hi;  // sequence, query block, key-tile range of the block
 };
 
 // Visible key interval [lo, hi] of query row i (sequence-relative) under the
@@ -40,15 +42,16 @@ __host__ __device__ __forceinline__ void row_key_interval(int i, int L_q, int L_
     }
 }
 
-// Key-tile range of query tile qt.  The intervals of consecutive rows have
-// non-decreasing ends and overlap or touch, so the union over the tile is the
-// interval of its first non-empty row to its last row.
-__host__ __device__ __forceinline__ void tile_key_range(int qt, int L_q, int L_k, bool causal,
-                                                        int window, int& kt_lo, int& kt_hi) {
+// Key-tile range of query rows [first, first + rows) clipped to L_q.  The
+// intervals of consecutive rows have non-decreasing ends and overlap or
+// touch, so the union over the rows is the interval of the first non-empty
+// row to the last row.  (0, 0) when no row sees a key.
+__host__ __device__ __forceinline__ void rows_key_range(int first, int rows, int L_q, int L_k,
+                                                        bool causal, int window, int& kt_lo,
+                                                        int& kt_hi) {
     kt_lo = kt_hi = 0;
     if (L_k <= 0) return;
-    const int first = qt * kBlockM;
-    const int last = min(L_q, first + kBlockM) - 1;
+    const int last = min(L_q, first + rows) - 1;
     if (last < first) return;
     // first row whose interval is non-empty: diag >= 0 when the band is bounded above
     int r0 = first;
@@ -67,8 +70,9 @@ __host__ __device__ __forceinline__ void tile_key_range(int qt, int L_q, int L_k
 
 // Workspace header written by the builder and read by the attention kernels.
 struct SchedHeader {
-    int n_tiles;  // number of valid entries in the sorted list
-    int pad[3];
+    int n_tiles;    // number of valid entries in the sorted list
+    int next_item;  // work counter of the persistent grid (zeroed by the builder)
+    int pad[2];
 };
 
 }  // namespace va

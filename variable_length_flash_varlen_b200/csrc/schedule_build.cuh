@@ -1,4 +1,4 @@
-// Device-side builder of the longest-first query-tile list (one CTA).
+// Device-side builder of the longest-first query-block list (one CTA).
 #pragma once
 
 #include "schedule.cuh"
@@ -57,12 +57,13 @@ build_schedule_kernel(const int* __restrict__ cu_q, const int* __restrict__ cu_k
     int local = 0;
     for (int b = tid; b < batch; b += blockDim.x) {
         const int Lq = cu_q[b + 1] - cu_q[b];
-        local += (Lq + kBlockM - 1) / kBlockM;
+        local += (Lq + kBlockQ - 1) / kBlockQ;
     }
     const int total = block_sum(local, red);
     if (total > capacity) {
         if (tid == 0) {
             hdr->n_tiles = 0;
+            hdr->next_item = 0;
             atomicOr(&g_va_status, kStatusScheduleOverflow);
         }
         return;
@@ -76,13 +77,13 @@ build_schedule_kernel(const int* __restrict__ cu_q, const int* __restrict__ cu_k
         if (b < batch) {
             Lq = cu_q[b + 1] - cu_q[b];
             Lk = cu_k[b + 1] - cu_k[b];
-            n = (Lq + kBlockM - 1) / kBlockM;
+            n = (Lq + kBlockQ - 1) / kBlockQ;
         }
         int chunk_total;
         const int first = carry + block_exclusive_scan(n, red, chunk_total);
         for (int qt = 0; qt < n; ++qt) {
             int lo, hi;
-            tile_key_range(qt, Lq, Lk, causal != 0, window, lo, hi);
+            rows_key_range(qt * kBlockQ, kBlockQ, Lq, Lk, causal != 0, window, lo, hi);
             const int e = first + qt;
             scratch[e] = TileEntry{b, qt, lo, hi};
             if (sort_in_smem) {
@@ -97,7 +98,10 @@ build_schedule_kernel(const int* __restrict__ cu_q, const int* __restrict__ cu_k
     if (!sort_in_smem) {
         // beyond the shared-memory sort capacity: enumeration order
         for (int e = tid; e < total; e += blockDim.x) out[e] = scratch[e];
-        if (tid == 0) hdr->n_tiles = total;
+        if (tid == 0) {
+            hdr->n_tiles = total;
+            hdr->next_item = 0;
+        }
         return;
     }
     int P = 1;
@@ -124,7 +128,10 @@ build_schedule_kernel(const int* __restrict__ cu_q, const int* __restrict__ cu_k
     for (int r = tid; r < total; r += blockDim.x) {
         out[r] = scratch[static_cast<int>(keys[r] & 0xFFFFFFFFull)];
     }
-    if (tid == 0) hdr->n_tiles = total;
+    if (tid == 0) {
+        hdr->n_tiles = total;
+        hdr->next_item = 0;
+    }
 }
 
 }  // namespace va

@@ -104,11 +104,11 @@ cudaError_t ws_alloc(void** p, size_t bytes, cudaStream_t stream) {
     return cudaMallocFromPoolAsync(p, bytes, g_dev[dev].pool, stream);
 }
 
-// 2-D bf16 view [rows][cols] (cols contiguous), box 64 x 128, 128-byte swizzle.
-int make_tile_map(CUtensorMap* map, const void* base, long long cols, long long rows) {
+// 2-D bf16 view [rows][cols] (cols contiguous), box 64 x box_rows, 128-byte swizzle.
+int make_tile_map(CUtensorMap* map, const void* base, long long cols, long long rows, int box_rows) {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-    cuuint32_t box[2] = {64, 128};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -156,7 +156,7 @@ int validate(const Args& a) {
 }
 
 int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
-    const long long tiles_per_seq = (a.max_q + va::kBlockM - 1) / va::kBlockM;
+    const long long tiles_per_seq = (a.max_q + va::kBlockQ - 1) / va::kBlockQ;
     const long long cap_ll = tiles_per_seq * a.batch;
     if (cap_ll * a.H >= INT_MAX) return fail(VA_ERR_UNSUPPORTED, "too many query tiles x heads");
     const int cap = static_cast<int>(cap_ll);
@@ -175,9 +175,9 @@ int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
     CUtensorMap tq, tk, tv;
     const long long rows_q = std::max(1ll, static_cast<long long>(a.batch) * a.max_q);
     const long long rows_k = std::max(1ll, static_cast<long long>(a.batch) * a.max_k);
-    if ((rc = make_tile_map(&tq, a.q, static_cast<long long>(a.H) * a.D, rows_q)) != VA_OK ||
-        (rc = make_tile_map(&tk, a.k, static_cast<long long>(a.H_kv) * a.D, rows_k)) != VA_OK ||
-        (rc = make_tile_map(&tv, a.v, static_cast<long long>(a.H_kv) * a.D, rows_k)) != VA_OK) {
+    if ((rc = make_tile_map(&tq, a.q, static_cast<long long>(a.H) * a.D, rows_q, va::kBlockM)) != VA_OK ||
+        (rc = make_tile_map(&tk, a.k, static_cast<long long>(a.H_kv) * a.D, rows_k, va::kBlockN)) != VA_OK ||
+        (rc = make_tile_map(&tv, a.v, static_cast<long long>(a.H_kv) * a.D, rows_k, va::kBlockN)) != VA_OK) {
         cudaFreeAsync(ws, stream);
         return rc;
     }
