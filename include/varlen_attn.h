@@ -107,6 +107,31 @@ int varlen_attention_fwd_host(const void* q, const void* k, const void* v,
                               int causal, int window, void* out, float* lse, void* stream);
 
 /*
+ * Same operation as varlen_attention_fwd (always on the tensor-core prefill
+ * path, which also serves single-query sequences) for callers that must not
+ * allocate device memory: code inside a framework or serving runtime that
+ * owns all device memory through its own allocator, or a latency-critical
+ * loop that may not reach cudaMalloc or a stream-ordered allocator.  There is
+ * no counterpart on the pages; it exists only for those callers.
+ *
+ * The call allocates nothing.  Its workspace is a static device array of
+ * 1 MiB per device (every GPU that loads the library keeps it until the
+ * process exits), enough for batch * ceil(max_seqlen_q / 256) <= 32760 query
+ * blocks; larger problems return VA_ERR_UNSUPPORTED with a message, and
+ * varlen_attention_fwd serves them.  The first call on a device performs a
+ * one-time set-up with that device current (kernel attributes and the device
+ * address of the static array); make that first call before any stream
+ * capture.  All calls on a device share the one array and every call rewrites
+ * what it reads, but calls whose work overlaps on the GPU (concurrent streams)
+ * race on it: order them on one stream or serialise them.
+ */
+int varlen_attention_fwd_noalloc(const void* q, const void* k, const void* v,
+                                 const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                 int batch, int num_heads, int num_kv_heads,
+                                 int max_seqlen_q, int max_seqlen_k, int head_dim,
+                                 int causal, int window, void* out, float* lse, void* stream);
+
+/*
  * The longest-first work list the prefill path builds from cu_seqlens
  * (device pointers), written to `tiles` (device int32 [capacity][4] =
  * {sequence, query block, first key tile, end key tile}) and its length to

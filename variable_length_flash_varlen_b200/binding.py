@@ -27,6 +27,7 @@ SIGNATURES = {
     "varlen_attention_fwd": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_fwd_ex": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _I, _I, _P]),
     "varlen_attention_fwd_host": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
+    "varlen_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_schedule": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P]),
     "varlen_attention_device_status": (_I, [ctypes.POINTER(ctypes.c_uint), _I]),
     "varlen_attention_last_error": (ctypes.c_char_p, []),
@@ -117,6 +118,27 @@ def varlen_attention_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         rc = lib.varlen_attention_fwd_ex(*args, int(path), int(decode_split_keys),
                                          _stream_ptr(stream))
     _check(rc)
+    return out, lse
+
+
+def varlen_attention_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                 cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                                 batch: int, num_heads: int, num_kv_heads: int,
+                                 max_seqlen_q: int, max_seqlen_k: int, head_dim: int,
+                                 causal: bool, window: int, out: torch.Tensor, lse: torch.Tensor,
+                                 stream: Optional[torch.cuda.Stream] = None):
+    """The allocation-free entry point: the caller passes out and lse; the
+    library's workspace is its static per-device scratch array."""
+    lib = load()
+    _check_inputs(q, k, v, cu_seqlens_q, cu_seqlens_k, num_heads, num_kv_heads, head_dim, "cuda")
+    if out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    if lse.shape != (q.shape[0], num_heads) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [total_q, num_heads] tensor")
+    _check(lib.varlen_attention_fwd_noalloc(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(),
+        batch, num_heads, num_kv_heads, max_seqlen_q, max_seqlen_k, head_dim, int(bool(causal)),
+        int(window), out.data_ptr(), lse.data_ptr(), _stream_ptr(stream)))
     return out, lse
 
 

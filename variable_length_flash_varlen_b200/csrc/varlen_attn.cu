@@ -284,6 +284,137 @@ int forward(const Args& a, int path, int split_keys, cudaStream_t stream) {
     return path == VA_PATH_DECODE ? run_decode(a, split_keys, stream) : run_prefill(a, *info, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Entry point without allocation.  Some callers must not reach any device
+// allocator: code running inside a framework or serving runtime that owns all
+// device memory through its own allocator, or a latency-critical loop that may
+// not call cudaMalloc or a stream-ordered allocator.  For them the prefill
+// path's workspace (the work-list header and two copies of the query-block
+// list) lives in a fixed static device array instead.
+
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;  // 1 MiB per device
+constexpr size_t kNoAllocHeaderBytes = 256;
+// query blocks the array can describe: header + scratch list + sorted list
+constexpr long long kNoAllocMaxBlocks =
+    static_cast<long long>((kNoAllocScratchBytes - kNoAllocHeaderBytes) / (2 * sizeof(va::TileEntry)));
+
+struct NoAllocState {
+    bool ready = false;
+    int num_sms = 0;
+    unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+};
+NoAllocState g_noalloc[kMaxDevices];
+
+}  // namespace
+
+// One copy per device that loads the library, held until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Once per device, with that device current: kernel attributes, the tensor-map
+// encoder and the device address of the static scratch array (in host code the
+// array's name is only a stand-in, not an address a kernel may be given).
+int noalloc_setup(NoAllocState*& st) {
+    int dev = 0;
+    VA_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return fail(VA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    st = &g_noalloc[dev];
+    if (st->ready) return VA_OK;
+    cudaDeviceProp prop;
+    VA_CUDA(cudaGetDeviceProperties(&prop, dev));
+    if (prop.major != 10)
+        return fail(VA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a",
+                    dev, prop.major, prop.minor);
+    if (!g_encode) {
+        cudaDriverEntryPointQueryResult q;
+        void* fn = nullptr;
+        VA_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+        if (q != cudaDriverEntryPointSuccess || !fn)
+            return fail(VA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::PrefillSmem<64>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::PrefillSmem<128>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::build_schedule_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::kSortCapacity * 8));
+    void* addr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
+    if (e != cudaSuccess || addr == nullptr)
+        return cuda_fail(e == cudaSuccess ? cudaErrorInvalidSymbol : e,
+                         "cudaGetSymbolAddress(g_noalloc_scratch)");
+    st->scratch = static_cast<unsigned char*>(addr);
+    st->num_sms = prop.multiProcessorCount;
+    st->ready = true;
+    return VA_OK;
+}
+
+int run_prefill_noalloc(const Args& a, cudaStream_t stream) {
+    const long long blocks = static_cast<long long>(a.batch) * ((a.max_q + va::kBlockQ - 1) / va::kBlockQ);
+    if (blocks > kNoAllocMaxBlocks)
+        return fail(VA_ERR_UNSUPPORTED,
+                    "batch x ceil(max_seqlen_q / %d) = %lld query blocks exceeds the %lld that the "
+                    "%zu-byte static scratch holds; use varlen_attention_fwd",
+                    va::kBlockQ, blocks, kNoAllocMaxBlocks, kNoAllocScratchBytes);
+    if (blocks * a.H >= INT_MAX) return fail(VA_ERR_UNSUPPORTED, "too many query blocks x heads");
+    NoAllocState* st = nullptr;
+    int rc = noalloc_setup(st);
+    if (rc != VA_OK) return rc;
+    const int cap = static_cast<int>(blocks);
+    int key_slots = 1;
+    while (key_slots < cap && key_slots < va::kSortCapacity) key_slots <<= 1;
+    const size_t list_bytes = static_cast<size_t>(cap) * sizeof(va::TileEntry);
+    auto* hdr = reinterpret_cast<va::SchedHeader*>(st->scratch);
+    auto* scratch = reinterpret_cast<va::TileEntry*>(st->scratch + kNoAllocHeaderBytes);
+    auto* tiles = reinterpret_cast<va::TileEntry*>(st->scratch + kNoAllocHeaderBytes + list_bytes);
+
+    CUtensorMap tq, tk, tv;
+    const long long rows_q = std::max(1ll, static_cast<long long>(a.batch) * a.max_q);
+    const long long rows_k = std::max(1ll, static_cast<long long>(a.batch) * a.max_k);
+    if ((rc = make_tile_map(&tq, a.q, static_cast<long long>(a.H) * a.D, rows_q, va::kBlockM)) != VA_OK ||
+        (rc = make_tile_map(&tk, a.k, static_cast<long long>(a.H_kv) * a.D, rows_k, va::kBlockN)) != VA_OK ||
+        (rc = make_tile_map(&tv, a.v, static_cast<long long>(a.H_kv) * a.D, rows_k, va::kBlockN)) != VA_OK)
+        return rc;
+    // the builder rewrites the whole header (count and work counter) and every
+    // list entry it hands out, so nothing left by the previous call is read
+    va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
+        a.cu_q, a.cu_k, a.batch, a.causal, a.window, cap, key_slots, scratch, tiles, hdr);
+    cudaError_t be = cudaGetLastError();
+    if (be != cudaSuccess) return cuda_fail(be, "schedule build launch");
+
+    va::PrefillParams p;
+    p.cu_q = a.cu_q;
+    p.cu_k = a.cu_k;
+    p.batch = a.batch;
+    p.H = a.H;
+    p.H_kv = a.H_kv;
+    p.causal = a.causal;
+    p.window = a.window;
+    p.tiles = tiles;
+    p.hdr = hdr;
+    p.tile_capacity = cap;
+    p.q = static_cast<const __nv_bfloat16*>(a.q);
+    p.k = static_cast<const __nv_bfloat16*>(a.k);
+    p.v = static_cast<const __nv_bfloat16*>(a.v);
+    p.out = static_cast<__nv_bfloat16*>(a.out);
+    p.lse = a.lse;
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)));
+    const int grid = static_cast<int>(std::min<long long>(st->num_sms, blocks * a.H));
+    if (a.D == 64)
+        va::prefill_fwd_kernel<64><<<grid, va::kPrefillThreads, va::PrefillSmem<64>::kAlloc, stream>>>(tq, tk, tv, p);
+    else
+        va::prefill_fwd_kernel<128><<<grid, va::kPrefillThreads, va::PrefillSmem<128>::kAlloc, stream>>>(tq, tk, tv, p);
+    cudaError_t le = cudaGetLastError();
+    if (le != cudaSuccess) return cuda_fail(le, "prefill launch");
+    return VA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -408,6 +539,20 @@ int varlen_attention_device_status(unsigned* status, int clear) {
         VA_CUDA(cudaMemcpyToSymbol(va::g_va_status, &zero, sizeof(unsigned)));
     }
     return VA_OK;
+}
+
+int varlen_attention_fwd_noalloc(const void* q, const void* k, const void* v,
+                                 const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                                 int num_heads, int num_kv_heads, int max_seqlen_q, int max_seqlen_k,
+                                 int head_dim, int causal, int window, void* out, float* lse,
+                                 void* stream) {
+    g_last_error[0] = 0;
+    Args a{q, k, v, cu_seqlens_q, cu_seqlens_k, batch, num_heads, num_kv_heads, max_seqlen_q,
+           max_seqlen_k, head_dim, causal ? 1 : 0, window, out, lse};
+    int rc = validate(a);
+    if (rc != VA_OK) return rc;
+    if (batch == 0 || max_seqlen_q == 0) return VA_OK;
+    return run_prefill_noalloc(a, static_cast<cudaStream_t>(stream));
 }
 
 const char* varlen_attention_last_error(void) { return g_last_error; }
