@@ -89,7 +89,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.reader = threading.Thread(target=self._read, daemon=True)
             self.reader.start()
@@ -319,8 +319,9 @@ def run_ours(args, world, rank, local):
 
     visible = os.environ.get("CUDA_VISIBLE_DEVICES")
     smi_index = int(visible.split(",")[local]) if visible and visible.split(",")[local].isdigit() else local
-    with ClockSampler(smi_index if not args.no_clock_sampler else None) as clk:
-        step_ms, outer_ms = time_device_steps(step, args.steps, args.warmup, flush, world, stream)
+    # clocks are sampled across all three timed loops (prefill, decode, end to end)
+    clk = ClockSampler(smi_index if not args.no_clock_sampler else None).__enter__()
+    step_ms, outer_ms = time_device_steps(step, args.steps, args.warmup, flush, world, stream)
     t_local = sum(step_ms) / 1e3
     t_max = max_over_ranks(t_local, world)
     total_flops = sum_over_ranks(flops * args.steps, world)
@@ -363,6 +364,7 @@ def run_ours(args, world, rank, local):
                                           wl.window, outh, lseh)
 
     e_ms, _ = time_device_steps(estep, args.steps, args.warmup, flush, world, stream)
+    clk.__exit__(None, None, None)
     e_max = max_over_ranks(sum(e_ms) / 1e3, world)
     e_value = total_flops / e_max / 1e12
     h2d = (q.numel() + k.numel() + v.numel()) * 2 + (len(wl.cu_q) + len(wl.cu_k)) * 4
