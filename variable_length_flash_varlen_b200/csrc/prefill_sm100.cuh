@@ -319,14 +319,18 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 }
                 mma_commit(&s_full[x]);
             };
-            auto issue_pv = [&](int x, int s, bool first) {
+            // O_x += P_x V.  Only the half's last PV of the item is committed to
+            // o_done (the epilogue waits for it); earlier ones need no barrier of
+            // their own: the S-ready commit of the next QK of the same half tracks
+            // every MMA issued before it, this PV included.
+            auto issue_pv = [&](int x, int s, bool first, bool last) {
                 const uint32_t vb = v_lo + ((s * L::kTileBytes) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk) {
                     mma_ts_lh<idesc_pv>(tmem + L::tmem_o(x), tmem + L::tmem_s(x) + kk * 8,
                                         vb + ((kk * 16 * 128) >> 4), v_hi, (!first || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(&o_done[x]);
+                if (last) mma_commit(&o_done[x]);
             };
 
             for (;;) {
@@ -366,7 +370,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         if (takes_part(it, x, kt)) {
                             if (!(ok = mbar_wait(&p_full[x], p_waits[x]++ & 1, abort_flag, status))) break;
                             tc_fence_after();
-                            issue_pv(x, s, first_pv[x]);
+                            issue_pv(x, s, first_pv[x], kt + 1 == it.hi_h[x]);
                             first_pv[x] = false;
                         }
                         if (has_next && takes_part(it, x, kt + 1)) {
@@ -498,9 +502,8 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 l = l * alpha + (((sums[0] + sums[1]) + (sums[2] + sums[3])) +
                                  ((sums[4] + sums[5]) + (sums[6] + sums[7])));
                 if (!first_tile) {
-                    // O_x must hold every earlier P V before it is rescaled
-                    if (!(ok = mbar_wait_warp(&o_done[x], o_waits++ & 1, abort_flag, status))) break;
-                    tc_fence_after();
+                    // O_x holds every earlier P V: they were issued before this tile's
+                    // QK, whose completion the S-ready barrier just observed
                     if (move) {
 #pragma unroll
                         for (int c = 0; c < D / 32; ++c) {
@@ -520,7 +523,8 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 if (lane == 0) mbar_arrive(&p_full[x]);
             }
             if (!ok) break;
-            // epilogue: wait for the last P V, then O / l and logsumexp
+            // epilogue: wait for the half's last P V (the only one committed to
+            // o_done), then O / l and logsumexp
             if (!(ok = mbar_wait_warp(&o_done[x], o_waits++ & 1, abort_flag, status))) break;
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
