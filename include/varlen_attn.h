@@ -82,8 +82,10 @@ int varlen_attention_fwd(const void* q, const void* k, const void* v,
 
 /*
  * Same as varlen_attention_fwd with the path forced (VA_PATH_*) and, for the
- * decode path, the number of keys per split (decode_split_keys in [32, 1024],
- * 0 = library default).  Used by tests that check path and split invariance.
+ * decode path, the number of keys per split (decode_split_keys in [32, 65536];
+ * 0 = library default: the largest of 4096, 2048, ..., 256 keys that still
+ * gives every SM at least eight work units, counted with max_seqlen_k).  Used
+ * by tests that check path and split invariance.
  */
 int varlen_attention_fwd_ex(const void* q, const void* k, const void* v,
                             const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,

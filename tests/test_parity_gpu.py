@@ -115,7 +115,7 @@ def test_host_buffer_entry_matches_device_entry():
 
 # --- decode path -------------------------------------------------------------------
 
-@pytest.mark.parametrize("split_keys", [32, 100, 448, 1024])
+@pytest.mark.parametrize("split_keys", [32, 100, 448, 1024, 5000])
 def test_decode_split_invariance(oracle_lib, split_keys):
     wl = workloads.named("decode", scale=1 / 32)
     q, k, v = workloads.make_qkv(wl)
@@ -135,6 +135,39 @@ def test_decode_equals_prefill_path_and_causal_noop(oracle_lib):
     wl_c = workloads.custom([1, 1, 0, 1, 1], [700, 1, 5, 0, 2000], 8, 2, 128, True, 0, seed=21)
     c = run_gpu(wl_c, q, k, v, path=binding.VA_PATH_DECODE)
     assert torch.equal(c[0], d[0]) and torch.equal(c[1], d[1])
+
+
+DECODE_EDGE = [
+    # lengths_k, H, H_kv, D, causal: GQA groups of 1, 6, 16 and 32 heads (the
+    # last spans two head groups of a KV head), D = 64, a packed K/V shorter
+    # than one 64-key tile, empty key sequences
+    ([40, 1, 63], 4, 4, 128, False),
+    ([900, 2100, 130, 4097], 12, 2, 64, False),
+    ([1500, 3000, 0], 32, 2, 128, False),
+    ([1500, 777], 64, 2, 128, True),
+    ([20, 0, 7], 8, 2, 64, True),
+]
+
+
+@pytest.mark.parametrize("case", DECODE_EDGE)
+def test_decode_edge_cases(oracle_lib, case):
+    Lk, H, Hkv, D, causal = case
+    wl = workloads.custom([1] * len(Lk), Lk, H, Hkv, D, causal, 0, seed=41)
+    q, k, v = workloads.make_qkv(wl)
+    ref_o, ref_l = oracle_all(oracle_lib, wl, q, k, v)
+    for split in (0, 64):
+        out, lse = run_gpu(wl, q, k, v, path=binding.VA_PATH_DECODE, split_keys=split)
+        compare(out, lse, ref_o, ref_l)
+
+
+def test_decode_large_scores(oracle_lib):
+    # scores spanning about +-40 move the running max on many tiles
+    wl = workloads.custom([1] * 3, [3000, 1700, 65], 8, 2, 128, False, 0, seed=43)
+    q, k, v = workloads.make_qkv(wl)
+    q = (q.float() * 6).to(torch.bfloat16)
+    out, lse = run_gpu(wl, q, k, v, path=binding.VA_PATH_DECODE, split_keys=1024)
+    ref_o, ref_l = oracle_all(oracle_lib, wl, q, k, v)
+    compare(out, lse, ref_o, ref_l)
 
 
 @pytest.mark.parametrize("W", [1, 300, 5000])

@@ -234,6 +234,35 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
            | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ------------------------------------------- warp-level tensor-core tiles --
+// Four 8x8 bf16 matrices from shared memory; lane i gives the address of row
+// (i & 7) of matrix (i >> 3).  Without .trans lane i receives, of each matrix,
+// row i/4, columns 2(i%4) and 2(i%4)+1; with .trans it receives that pair from
+// column i/4 (rows 2(i%4), 2(i%4)+1).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// d[16x8] += a[16x16] b[16x8], bf16 inputs, f32 accumulate.  With g = lane/4,
+// t = lane%4: a = {(g, 2t..2t+1), (g+8, 2t..), (g, 2t+8..), (g+8, 2t+8..)},
+// b = {(k 2t..2t+1, n g), (k 2t+8.., n g)}, d = {(g, 2t), (g, 2t+1),
+// (g+8, 2t), (g+8, 2t+1)}; a pair holds its lower column in the low half.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // ------------------------------------------------------------------ math --
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;

@@ -83,6 +83,18 @@ int device_setup(int& dev, DeviceInfo*& info) {
     VA_CUDA(cudaFuncSetAttribute(va::build_schedule_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  va::kSortCapacity * 8));
+    VA_CUDA(cudaFuncSetAttribute(va::decode_stream_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::DecodeSmem<64>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::decode_stream_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::DecodeSmem<128>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::decode_stream_kernel<64>,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared));
+    VA_CUDA(cudaFuncSetAttribute(va::decode_stream_kernel<128>,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared));
     cudaMemPoolProps props = {};
     props.allocType = cudaMemAllocationTypePinned;
     props.handleTypes = cudaMemHandleTypeNone;
@@ -219,21 +231,41 @@ int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
     return VA_OK;
 }
 
-int run_decode(const Args& a, int split_keys, cudaStream_t stream) {
-    int chunk = split_keys > 0 ? split_keys : va::kDecodeMaxChunk;
-    if (chunk < 32 || chunk > va::kDecodeMaxChunk)
-        return fail(VA_ERR_INVALID_ARG, "decode_split_keys must be in [32, %d] (got %d)",
-                    va::kDecodeMaxChunk, split_keys);
-    const int n_split_max = std::max(1, (a.max_k + chunk - 1) / chunk);
+int run_decode(const Args& a, const DeviceInfo& dev, int split_keys, cudaStream_t stream) {
+    if (split_keys != 0 && (split_keys < 32 || split_keys > 65536))
+        return fail(VA_ERR_INVALID_ARG, "decode_split_keys must be in [32, 65536] (got %d)", split_keys);
     const int G = a.H / a.H_kv;
-    const int groups = a.H_kv * ((G + va::kDecodeHeads - 1) / va::kDecodeHeads);
-    if (groups > 65535 || n_split_max > 65535)
-        return fail(VA_ERR_UNSUPPORTED, "decode grid too large (kv groups %d, splits %d)", groups,
-                    n_split_max);
+    const long long groups = static_cast<long long>(a.H_kv) * ((G + va::kDecodeHeads - 1) / va::kDecodeHeads);
+    int chunk = split_keys;
+    if (chunk == 0) {
+        // fewest splits that still give every SM several units to claim
+        const long long want = static_cast<long long>(va::kDecodeUnitsPerSm) * dev.num_sms;
+        chunk = va::kDecodeMaxDefaultChunk;
+        while (chunk > va::kDecodeMinDefaultChunk &&
+               groups * a.batch * ((a.max_k + chunk - 1) / chunk) < want)
+            chunk /= 2;
+    }
+    const int n_split_max = std::max(1, (a.max_k + chunk - 1) / chunk);
+    const long long n_units = groups * a.batch * n_split_max;
+    if (n_units >= INT_MAX) return fail(VA_ERR_UNSUPPORTED, "decode work units beyond int32");
     const size_t slots = static_cast<size_t>(a.batch) * a.H * n_split_max;
-    char* ws = nullptr;
+    const size_t hdr = 256;
     const size_t o_bytes = slots * a.D * sizeof(float);
-    VA_CUDA(ws_alloc(reinterpret_cast<void**>(&ws), o_bytes + slots * 2 * sizeof(float), stream));
+    char* ws = nullptr;
+    VA_CUDA(ws_alloc(reinterpret_cast<void**>(&ws), hdr + o_bytes + slots * 2 * sizeof(float), stream));
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int), stream);
+    if (e != cudaSuccess) {
+        cudaFreeAsync(ws, stream);
+        return cuda_fail(e, "cudaMemsetAsync (decode work counter)");
+    }
+    CUtensorMap tk, tv;
+    const long long rows_k = std::max(1ll, static_cast<long long>(a.batch) * a.max_k);
+    int rc;
+    if ((rc = make_tile_map(&tk, a.k, static_cast<long long>(a.H_kv) * a.D, rows_k, va::kDecodeTileKeys)) != VA_OK ||
+        (rc = make_tile_map(&tv, a.v, static_cast<long long>(a.H_kv) * a.D, rows_k, va::kDecodeTileKeys)) != VA_OK) {
+        cudaFreeAsync(ws, stream);
+        return rc;
+    }
 
     va::DecodeParams p;
     p.cu_q = a.cu_q;
@@ -246,19 +278,21 @@ int run_decode(const Args& a, int split_keys, cudaStream_t stream) {
     p.q = static_cast<const __nv_bfloat16*>(a.q);
     p.k = static_cast<const __nv_bfloat16*>(a.k);
     p.v = static_cast<const __nv_bfloat16*>(a.v);
-    p.part_o = reinterpret_cast<float*>(ws);
-    p.part_ml = reinterpret_cast<float*>(ws + o_bytes);
+    p.counter = reinterpret_cast<int*>(ws);
+    p.part_o = reinterpret_cast<float*>(ws + hdr);
+    p.part_ml = reinterpret_cast<float*>(ws + hdr + o_bytes);
     p.n_split_max = n_split_max;
     p.chunk = chunk;
+    p.n_units = static_cast<int>(n_units);
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)));
     p.out = static_cast<__nv_bfloat16*>(a.out);
     p.lse = a.lse;
-    dim3 grid(a.batch, groups, n_split_max);
+    const int grid = static_cast<int>(std::min<long long>(dev.num_sms, n_units));
     if (a.D == 64) {
-        va::decode_split_kernel<64><<<grid, va::kDecodeThreads, 0, stream>>>(p);
+        va::decode_stream_kernel<64><<<grid, va::kDecodeThreads, va::DecodeSmem<64>::kAlloc, stream>>>(tk, tv, p);
         va::decode_combine_kernel<64><<<a.batch * a.H, 64, 0, stream>>>(p);
     } else {
-        va::decode_split_kernel<128><<<grid, va::kDecodeThreads, 0, stream>>>(p);
+        va::decode_stream_kernel<128><<<grid, va::kDecodeThreads, va::DecodeSmem<128>::kAlloc, stream>>>(tk, tv, p);
         va::decode_combine_kernel<128><<<a.batch * a.H, 128, 0, stream>>>(p);
     }
     cudaError_t le = cudaGetLastError();
@@ -281,7 +315,7 @@ int forward(const Args& a, int path, int split_keys, cudaStream_t stream) {
     int dev;
     DeviceInfo* info;
     if ((rc = device_setup(dev, info)) != VA_OK) return rc;
-    return path == VA_PATH_DECODE ? run_decode(a, split_keys, stream) : run_prefill(a, *info, stream);
+    return path == VA_PATH_DECODE ? run_decode(a, *info, split_keys, stream) : run_prefill(a, *info, stream);
 }
 
 // ---------------------------------------------------------------------------
