@@ -70,8 +70,9 @@ struct PrefillSmem {
     // q_full[2], q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
     // o_done[2], item_full[2], item_empty[2]
     static constexpr int kNumBars = 3 + 4 * kStages + 10;
-    static constexpr int kMisc = kBar + kNumBars * 8;
-    static constexpr int kBytes = kMisc + 16;  // tmem slot, abort flag, item ring[2]
+    static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag, item ring[2]
+    static constexpr int kItems = kMisc + 16;          // the ring's decoded items [2]
+    static constexpr int kBytes = kItems + 2 * 64;
     // slack for 1024-byte alignment; never below 120 KB so that at most one CTA
     // (and one 512-column tensor-memory allocation) is resident per SM
     static constexpr int kAlloc = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
@@ -87,6 +88,7 @@ struct Item {
     int lo, hi;           // key-tile range of the block (union of the halves)
     int lo_h[2], hi_h[2]; // key-tile range of each 128-row half
 };
+static_assert(sizeof(Item) <= 64, "an item must fit its 64-byte ring slot");
 
 __device__ __forceinline__ void decode_item(const PrefillParams& p, int idx, int group, Item& it) {
     const TileEntry te = p.tiles[idx / p.H];
@@ -183,6 +185,9 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     volatile int* item_ring = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [2]
+    // the producer decodes each item once (cu_seqlens and the tile list are
+    // global-memory reads) and publishes it here next to its index
+    Item* item_slot = reinterpret_cast<Item*>(smem + L::kItems);                   // [2]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -237,17 +242,18 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 idx = t < n_items ? t : -1;
             }
             idx = __shfl_sync(0xffffffffu, idx, 0);
+            Item it;
+            if (idx >= 0) decode_item(p, idx, group, it);
             if (!(ok = mbar_wait_warp(&item_empty[ring & 1], ((ring >> 1) & 1) ^ 1, abort_flag, status)))
                 break;
             if (lane == 0) {
                 item_ring[ring & 1] = idx;
-                mbar_arrive(&item_full[ring & 1]);
+                if (idx >= 0) item_slot[ring & 1] = it;
+                mbar_arrive(&item_full[ring & 1]);  // release: the slot's contents are visible
             }
             __syncwarp();
             ++ring;
             if (idx < 0) break;
-            Item it;
-            decode_item(p, idx, group, it);
             if (it.hi <= it.lo) continue;
             if (!(ok = mbar_wait_warp(q_empty, (items_done & 1) ^ 1, abort_flag, status))) break;
             ++items_done;
@@ -336,11 +342,11 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             for (;;) {
                 if (!(ok = mbar_wait(&item_full[ring & 1], (ring >> 1) & 1, abort_flag, status))) break;
                 const int idx = item_ring[ring & 1];
+                Item it;
+                if (idx >= 0) it = item_slot[ring & 1];
                 mbar_arrive(&item_empty[ring & 1]);
                 ++ring;
                 if (idx < 0) break;
-                Item it;
-                decode_item(p, idx, group, it);
                 if (it.hi <= it.lo) continue;
                 const int n = it.hi - it.lo;
                 for (int x = 0; x < 2 && ok; ++x) {
@@ -416,12 +422,12 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         for (;;) {
             if (!(ok = mbar_wait_warp(&item_full[ring & 1], (ring >> 1) & 1, abort_flag, status))) break;
             const int idx = item_ring[ring & 1];
+            Item it;
+            if (idx >= 0) it = item_slot[ring & 1];
             __syncwarp();
             if (lane == 0) mbar_arrive(&item_empty[ring & 1]);
             ++ring;
             if (idx < 0) break;
-            Item it;
-            decode_item(p, idx, group, it);
             const int i = it.qb * kBlockQ + x * kBlockM + row_in_tile;
             const bool row_valid = i < it.L_q;
             int lo, hi;
@@ -528,21 +534,25 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             if (!(ok = mbar_wait_warp(&o_done[x], o_waits++ & 1, abort_flag, status))) break;
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            {
+                // every column block in flight before a single wait
+                uint32_t r[D / 32][32];
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(obase + c * 32, r);
+                for (int c = 0; c < D / 32; ++c) tmem_ld32(obase + c * 32, r[c]);
                 tmem_wait_ld();
                 if (row_valid) {
-                    uint4* o4 = reinterpret_cast<uint4*>(p.out + out_row * D + c * 32);
+                    uint4* o4 = reinterpret_cast<uint4*>(p.out + out_row * D);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(r[8 * e + 0]) * inv_l, __uint_as_float(r[8 * e + 1]) * inv_l);
-                        w.y = pack_bf16x2(__uint_as_float(r[8 * e + 2]) * inv_l, __uint_as_float(r[8 * e + 3]) * inv_l);
-                        w.z = pack_bf16x2(__uint_as_float(r[8 * e + 4]) * inv_l, __uint_as_float(r[8 * e + 5]) * inv_l);
-                        w.w = pack_bf16x2(__uint_as_float(r[8 * e + 6]) * inv_l, __uint_as_float(r[8 * e + 7]) * inv_l);
-                        o4[e] = w;
+                    for (int c = 0; c < D / 32; ++c) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            uint4 w;
+                            w.x = pack_bf16x2(__uint_as_float(r[c][8 * e + 0]) * inv_l, __uint_as_float(r[c][8 * e + 1]) * inv_l);
+                            w.y = pack_bf16x2(__uint_as_float(r[c][8 * e + 2]) * inv_l, __uint_as_float(r[c][8 * e + 3]) * inv_l);
+                            w.z = pack_bf16x2(__uint_as_float(r[c][8 * e + 4]) * inv_l, __uint_as_float(r[c][8 * e + 5]) * inv_l);
+                            w.w = pack_bf16x2(__uint_as_float(r[c][8 * e + 6]) * inv_l, __uint_as_float(r[c][8 * e + 7]) * inv_l);
+                            o4[c * 4 + e] = w;
+                        }
                     }
                 }
             }
