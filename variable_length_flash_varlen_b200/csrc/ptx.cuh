@@ -78,38 +78,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Same contract as mbar_wait, polling with the non-blocking test_wait: for a
-// short wait on the critical path, where a thread suspended inside try_wait
-// has been measured to resume a few hundred cycles after the phase completes.
-__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                               unsigned* status) {
-    if (mbar_test_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_timer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_test_wait(bar, parity)) return true;
-        if ((it & 255u) == 0) {
-            if (*abort) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
-                *abort = 1;
-                atomicOr(status, kStatusWaitTimeout);
-                return false;
-            }
-        }
-    }
-}
-
 // Warp-uniform wait: lane 0 waits, the verdict is broadcast, so every lane of
 // the warp leaves with the same result (the warp then stays converged for the
 // .sync.aligned tcgen05 instructions and warp collectives that follow).  Must
