@@ -67,9 +67,9 @@ struct PrefillSmem {
     static constexpr int kK = kQ + 2 * kTileBytes;
     static constexpr int kV = kK + kStages * kTileBytes;
     static constexpr int kBar = kV + kStages * kTileBytes;
-    // q_full[2], q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
-    // o_done[2], item_full[2], item_empty[2]
-    static constexpr int kNumBars = 3 + 4 * kStages + 10;
+    // q_full[2], q_empty, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_half[2],
+    // p_full[2], o_done[2], item_full[2], item_empty[2]
+    static constexpr int kNumBars = 3 + 4 * kStages + 12;
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag, item ring[2]
     static constexpr int kItems = kMisc + 16;          // the ring's decoded items [2]
     static constexpr int kBytes = kItems + 2 * 64;
@@ -178,7 +178,8 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     uint64_t* v_full = k_empty + kStages;
     uint64_t* v_empty = v_full + kStages;
     uint64_t* s_full = v_empty + kStages;  // [2]
-    uint64_t* p_full = s_full + 2;         // [2]
+    uint64_t* p_half = s_full + 2;         // [2], P of the tile's first 64 keys stored
+    uint64_t* p_full = p_half + 2;         // [2], all of P stored
     uint64_t* o_done = p_full + 2;         // [2]
     uint64_t* item_full = o_done + 2;      // [2]
     uint64_t* item_empty = item_full + 2;  // [2]
@@ -195,6 +196,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         for (int x = 0; x < 2; ++x) {
             mbar_init(&q_full[x], 1);
             mbar_init(&s_full[x], 1);
+            mbar_init(&p_half[x], 4);
             mbar_init(&p_full[x], 4);
             mbar_init(&o_done[x], 1);
             mbar_init(&item_full[x], 1);
@@ -329,10 +331,12 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             // o_done (the epilogue waits for it); earlier ones need no barrier of
             // their own: the S-ready commit of the next QK of the same half tracks
             // every MMA issued before it, this PV included.
-            auto issue_pv = [&](int x, int s, bool first, bool last) {
+            // Keys [64 part, 64 part + 64) of the tile (the part-th half of P).
+            auto issue_pv = [&](int x, int s, bool first, bool last, int part) {
                 const uint32_t vb = v_lo + ((s * L::kTileBytes) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                for (int k4 = 0; k4 < kBlockN / 32; ++k4) {
+                    const int kk = part * (kBlockN / 32) + k4;
                     mma_ts_lh<idesc_pv>(tmem + L::tmem_o(x), tmem + L::tmem_s(x) + kk * 8,
                                         vb + ((kk * 16 * 128) >> 4), v_hi, (!first || kk > 0) ? 1u : 0u);
                 }
@@ -374,9 +378,13 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     if (!(ok = mbar_wait(&v_full[s], (kv_j / kStages) & 1, abort_flag, status))) break;
                     for (int x = 0; x < 2 && ok; ++x) {
                         if (takes_part(it, x, kt)) {
-                            if (!(ok = mbar_wait(&p_full[x], p_waits[x]++ & 1, abort_flag, status))) break;
+                            const uint32_t pw = p_waits[x]++ & 1;
+                            if (!(ok = mbar_wait(&p_half[x], pw, abort_flag, status))) break;
                             tc_fence_after();
-                            issue_pv(x, s, first_pv[x], kt + 1 == it.hi_h[x]);
+                            issue_pv(x, s, first_pv[x], false, 0);
+                            if (!(ok = mbar_wait(&p_full[x], pw, abort_flag, status))) break;
+                            tc_fence_after();
+                            issue_pv(x, s, first_pv[x], kt + 1 == it.hi_h[x], 1);
                             first_pv[x] = false;
                         }
                         if (has_next && takes_part(it, x, kt + 1)) {
@@ -490,8 +498,10 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     m_ref = m_cand;
                 }
                 const float m_sub = (m_ref == -INFINITY) ? 0.f : m_ref;
-                // P = 2^(s * scale_log2 - m_ref) as bf16 pairs into S_x, 32 columns at a
-                // time.  S_x's previous P was consumed by the PV issued before this QK.
+                // P = 2^(s * scale_log2 - m_ref) as bf16 pairs into S_x, 32 columns (64
+                // keys) at a time; the first 64 keys are handed over on their own so
+                // their PV starts while the second half is computed.  S_x's previous P
+                // was consumed by the PV issued before this QK.
                 float sums[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -504,25 +514,30 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         pk[c / 2] = pack_bf16x2(p0, p1);
                     }
                     tmem_st32(sbase + half * 32, pk);
+                    if (half == 0) {
+                        if (!first_tile && move) {
+                            // O_x holds every earlier P V: they were issued before this
+                            // tile's QK, whose completion the S-ready barrier observed.
+                            // Rescale it before any P of this tile reaches the MMA warp.
+#pragma unroll
+                            for (int c = 0; c < D / 32; ++c) {
+                                uint32_t r[32];
+                                tmem_ld32(obase + c * 32, r);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int e = 0; e < 32; ++e)
+                                    r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                                tmem_st32(obase + c * 32, r);
+                            }
+                        }
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&p_half[x]);
+                    }
                 }
                 l = l * alpha + (((sums[0] + sums[1]) + (sums[2] + sums[3])) +
                                  ((sums[4] + sums[5]) + (sums[6] + sums[7])));
-                if (!first_tile) {
-                    // O_x holds every earlier P V: they were issued before this tile's
-                    // QK, whose completion the S-ready barrier just observed
-                    if (move) {
-#pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t r[32];
-                            tmem_ld32(obase + c * 32, r);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                            tmem_st32(obase + c * 32, r);
-                        }
-                    }
-                }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
