@@ -49,10 +49,19 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+# Sources each kernel is compiled from (the launch code in varlen_attn.cu
+# included), so a recorded traffic figure goes stale only when its own kernel
+# changes.
+KERNEL_SOURCES = {
+    "prefill_fwd_kernel": ("prefill_sm100.cuh", "schedule.cuh", "ptx.cuh", "status.cuh", "varlen_attn.cu"),
+    "decode_stream_kernel": ("decode.cuh", "schedule.cuh", "ptx.cuh", "status.cuh", "varlen_attn.cu"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "variable_length_flash_varlen_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -67,7 +76,7 @@ def recorded_traffic(kernel: str, workload: str):
     with open(path) as f:
         rec = json.load(f)
     e = rec.get(kernel, {}).get(workload)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("bytes_per_launch")
 
