@@ -472,11 +472,15 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 }
                 const int key0 = kt * kBlockN;
                 if (!(warp_lo <= key0 && key0 + kBlockN - 1 <= warp_hi)) {
+                    // column c is visible iff lo <= key0 + c <= hi: one unsigned range
+                    // check per element against this row's bounds relative to the tile
+                    // (a row that sees no key gets an offset no column reaches)
+                    const bool any = hi >= lo;
+                    const int c_lo = any ? lo - key0 : (1 << 30);
+                    const unsigned span = any ? static_cast<unsigned>(hi - lo) : 0u;
 #pragma unroll
-                    for (int c = 0; c < kBlockN; ++c) {
-                        const int kj = key0 + c;
-                        s[c] = (kj >= lo && kj <= hi) ? s[c] : -INFINITY;
-                    }
+                    for (int c = 0; c < kBlockN; ++c)
+                        s[c] = (static_cast<unsigned>(c - c_lo) <= span) ? s[c] : -INFINITY;
                 }
                 // row max as a tree (short dependency chains)
                 float mv[8];
