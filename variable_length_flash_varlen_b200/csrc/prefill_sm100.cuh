@@ -72,7 +72,9 @@ struct PrefillSmem {
     static constexpr int kNumBars = 3 + 4 * kStages + 12;
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag, item ring[2]
     static constexpr int kItems = kMisc + 16;          // the ring's decoded items [2]
-    static constexpr int kBytes = kItems + 2 * 64;
+    // epilogue staging, per softmax warp 32 rows x 64 bytes (one 32-column block of O)
+    static constexpr int kStage = (kItems + 2 * 64 + 15) & ~15;
+    static constexpr int kBytes = kStage + 8 * 2048;
     // slack for 1024-byte alignment; never below 120 KB so that at most one CTA
     // (and one 512-column tensor-memory allocation) is resident per SM
     static constexpr int kAlloc = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
@@ -559,20 +561,35 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) tmem_ld32(obase + c * 32, r[c]);
                 tmem_wait_ld();
-                if (row_valid) {
-                    uint4* o4 = reinterpret_cast<uint4*>(p.out + out_row * D);
+                // Through a per-warp shared-memory slice, one 32-column block at a time,
+                // so that each global store instruction writes eight rows x 64
+                // contiguous bytes instead of 16 bytes of 32 different rows.  The
+                // 16-byte chunk e of slice row r sits at position e ^ ((r >> 1) & 3):
+                // both the row-per-lane writes and the 8-row reads are conflict-free.
+                uint8_t* stage = smem + L::kStage + warp * 2048;
+                const int row_base = x * kBlockM + quarter * 32;  // first tile row of this warp
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < D / 32; ++c) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            uint4 w;
-                            w.x = pack_bf16x2(__uint_as_float(r[c][8 * e + 0]) * inv_l, __uint_as_float(r[c][8 * e + 1]) * inv_l);
-                            w.y = pack_bf16x2(__uint_as_float(r[c][8 * e + 2]) * inv_l, __uint_as_float(r[c][8 * e + 3]) * inv_l);
-                            w.z = pack_bf16x2(__uint_as_float(r[c][8 * e + 4]) * inv_l, __uint_as_float(r[c][8 * e + 5]) * inv_l);
-                            w.w = pack_bf16x2(__uint_as_float(r[c][8 * e + 6]) * inv_l, __uint_as_float(r[c][8 * e + 7]) * inv_l);
-                            o4[c * 4 + e] = w;
+                    for (int e = 0; e < 4; ++e) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(r[c][8 * e + 0]) * inv_l, __uint_as_float(r[c][8 * e + 1]) * inv_l);
+                        w.y = pack_bf16x2(__uint_as_float(r[c][8 * e + 2]) * inv_l, __uint_as_float(r[c][8 * e + 3]) * inv_l);
+                        w.z = pack_bf16x2(__uint_as_float(r[c][8 * e + 4]) * inv_l, __uint_as_float(r[c][8 * e + 5]) * inv_l);
+                        w.w = pack_bf16x2(__uint_as_float(r[c][8 * e + 6]) * inv_l, __uint_as_float(r[c][8 * e + 7]) * inv_l);
+                        *reinterpret_cast<uint4*>(stage + lane * 64 + ((e ^ ((lane >> 1) & 3)) << 4)) = w;
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int rr = i * 8 + (lane >> 2), ch = lane & 3;
+                        const uint4 v = *reinterpret_cast<const uint4*>(stage + rr * 64 + ((ch ^ ((rr >> 1) & 3)) << 4));
+                        if (it.qb * kBlockQ + row_base + rr < it.L_q) {
+                            const size_t orow = static_cast<size_t>(it.q_row0 + row_base + rr) * p.H + it.h;
+                            *reinterpret_cast<uint4*>(p.out + orow * D + c * 32 + ch * 8) = v;
                         }
                     }
+                    __syncwarp();
                 }
             }
             if (row_valid) {
