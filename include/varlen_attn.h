@@ -154,6 +154,18 @@ int varlen_attention_schedule(const int32_t* cu_seqlens_q, const int32_t* cu_seq
  */
 int varlen_attention_device_status(unsigned* status, int clear);
 
+/*
+ * Self-test of the failure path (for tests; no fault or hang is involved).
+ * Launches on `stream` a one-thread kernel that waits, through the same
+ * bounded barrier wait every kernel of the library uses, on a barrier phase
+ * that nothing completes.  The wait gives up after its limit (2 s of device
+ * time), raises VA_STATUS_WAIT_TIMEOUT in the device status word and the
+ * kernel returns normally, writing 1 to *gave_up (device int32; 0 would mean
+ * the wait was satisfied).  The context stays usable afterwards.
+ * Returns VA_ERR_INVALID_ARG for a NULL gave_up, VA_ERR_CUDA if the launch fails.
+ */
+int varlen_attention_selftest_wait_timeout(int32_t* gave_up, void* stream);
+
 /* Message for the last non-VA_OK return on this host thread ("" if none). */
 const char* varlen_attention_last_error(void);
 

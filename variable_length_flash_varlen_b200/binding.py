@@ -30,6 +30,7 @@ SIGNATURES = {
     "varlen_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_schedule": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P]),
     "varlen_attention_device_status": (_I, [ctypes.POINTER(ctypes.c_uint), _I]),
+    "varlen_attention_selftest_wait_timeout": (_I, [_P, _P]),
     "varlen_attention_last_error": (ctypes.c_char_p, []),
     "varlen_attention_version": (_I, []),
 }
@@ -180,3 +181,12 @@ def device_status(clear: bool = True) -> int:
     st = ctypes.c_uint(0)
     _check(load().varlen_attention_device_status(ctypes.byref(st), int(clear)))
     return st.value
+
+
+def selftest_wait_timeout(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Run the failure-path probe (about 2 s of device time); returns its verdict
+    (1 = the bounded wait gave up).  Read the raised bit with device_status()."""
+    gave_up = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    _check(load().varlen_attention_selftest_wait_timeout(gave_up.data_ptr(), _stream_ptr(stream)))
+    (stream or torch.cuda.current_stream()).synchronize()
+    return int(gave_up.item())

@@ -18,6 +18,24 @@
 #include "schedule_build.cuh"
 #include "varlen_attn.h"
 
+namespace va {
+
+// Failure-path probe: one thread waits, through the bounded wait every kernel
+// of the library uses, on a barrier phase that nothing completes (no thread
+// arrives on it).  The wait gives up after its limit, raises the timeout bit
+// in the status word and the kernel returns normally.
+__global__ void wait_timeout_probe_kernel(int32_t* gave_up) {
+    __shared__ uint64_t bar;
+    __shared__ volatile int abort_flag;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+    *gave_up = mbar_wait(&bar, 0, &abort_flag, &g_va_status) ? 0 : 1;
+}
+
+}  // namespace va
+
 namespace {
 
 thread_local char g_last_error[512] = "";
@@ -587,6 +605,14 @@ int varlen_attention_fwd_noalloc(const void* q, const void* k, const void* v,
     if (rc != VA_OK) return rc;
     if (batch == 0 || max_seqlen_q == 0) return VA_OK;
     return run_prefill_noalloc(a, static_cast<cudaStream_t>(stream));
+}
+
+int varlen_attention_selftest_wait_timeout(int32_t* gave_up, void* stream) {
+    g_last_error[0] = 0;
+    if (!gave_up) return fail(VA_ERR_INVALID_ARG, "gave_up is NULL");
+    va::wait_timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(gave_up);
+    VA_CUDA(cudaGetLastError());
+    return VA_OK;
 }
 
 const char* varlen_attention_last_error(void) { return g_last_error; }
