@@ -328,7 +328,7 @@ def run_ours(args, world, rank, local):
 
     visible = os.environ.get("CUDA_VISIBLE_DEVICES")
     smi_index = int(visible.split(",")[local]) if visible and visible.split(",")[local].isdigit() else local
-    # clocks are sampled across all three timed loops (prefill, decode, end to end)
+    # clocks are sampled across all timed loops (prefill, decode, chunked prefill, end to end)
     clk = ClockSampler(smi_index if not args.no_clock_sampler else None).__enter__()
     step_ms, outer_ms = time_device_steps(step, args.steps, args.warmup, flush, world, stream)
     t_local = sum(step_ms) / 1e3
@@ -359,6 +359,26 @@ def run_ours(args, world, rank, local):
     dbytes = accounting.decode_bytes(dwl)
     d_value = sum_over_ranks(dbytes * args.steps, world) / d_max / 1e9
     del dqd, dkd, dvd, outd, lsed
+
+    # ---- chunked prefill: new query chunks after cached prefixes (L_q < L_k, causal)
+    cwl = workloads.named("chunked_prefill", seed=workloads.WORKLOAD_SEEDS["chunked_prefill"] + rank)
+    qc, kc, vc = workloads.make_qkv(cwl)
+    dqc, dkc, dvc = qc.to(dev), kc.to(dev), vc.to(dev)
+    cqc = torch.tensor(cwl.cu_q, dtype=torch.int32, device=dev)
+    ckc = torch.tensor(cwl.cu_k, dtype=torch.int32, device=dev)
+    outc = torch.empty_like(dqc)
+    lsec = torch.empty(cwl.total_q, cwl.H, dtype=torch.float32, device=dev)
+
+    def cstep():
+        binding.varlen_attention_fwd(dqc, dkc, dvc, cqc, ckc, cwl.batch, cwl.H, cwl.H_kv,
+                                     cwl.max_seqlen_q, cwl.max_seqlen_k, cwl.D, cwl.causal,
+                                     cwl.window, out=outc, lse=lsec)
+
+    c_ms, _ = time_device_steps(cstep, args.steps, args.warmup, flush, world, stream)
+    c_max = max_over_ranks(sum(c_ms) / 1e3, world)
+    cflops = accounting.attention_flops(cwl)
+    c_value = sum_over_ranks(cflops * args.steps, world) / c_max / 1e12
+    del dqc, dkc, dvc, outc, lsec, qc, kc, vc
 
     # ---- end to end through the host-buffer entry point (pinned memory)
     qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
@@ -411,6 +431,12 @@ def run_ours(args, world, rank, local):
                                 "kernel": "decode_stream_kernel<128> (+ combine and counter reset, same call)",
                                 "traffic": recorded_traffic("decode_stream_kernel", "decode")},
                    "gpu_launches": 2 * args.steps},
+        "chunked_prefill": {**cwl.describe(), "value": c_value, "unit": "TFLOP/s",
+                            "ms_per_step": c_max / args.steps * 1e3, "flops_per_step_per_gpu": cflops,
+                            "roofline": {"bound": "tensor", "achieved": c_value / world, "peak": peak,
+                                         "unit": "TFLOP/s", "frac": c_value / world / peak,
+                                         "peak_kind": f"{peak_kind} bf16 burst"},
+                            "gpu_launches": 2 * args.steps},
         "e2e": {"value": e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,

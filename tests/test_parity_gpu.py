@@ -27,7 +27,7 @@ def _lib():
 # --- reduced-size versions of the named workloads (full comparison) ------------
 
 REDUCED = [("worked_example", 1.0), ("mha_noncausal", 0.15), ("gqa_causal", 0.05),
-           ("sliding_window", 1 / 32), ("decode", 1 / 32)]
+           ("sliding_window", 1 / 32), ("decode", 1 / 32), ("chunked_prefill", 0.1)]
 
 
 @pytest.mark.parametrize("name,scale", REDUCED)

@@ -21,6 +21,10 @@ Named workloads (all bf16, Q/K/V ~ N(0, 1), softmax scale 1/sqrt(D)):
   sliding_window   4 sequences of 32768, window 4096, causal, H=32, H_kv=8, D=128
   decode           128 sequences, q length 1, k lengths uniform-int in
                    [1024, 32768], non-causal, H=32, H_kv=8, D=128
+  chunked_prefill  32 sequences, each a new chunk of q length uniform-int in
+                   [128, 1024] appended to a cached prefix of uniform-int
+                   [0, 8192] keys (k length = prefix + chunk), causal with the
+                   diagonal at the end of the keys, H=32, H_kv=8, D=128
 Lengths come from random.Random(seed); Q, K, V (in that order) from a torch
 CPU generator seeded with the same seed, drawn in fixed-size chunks.
 """
@@ -41,6 +45,7 @@ WORKLOAD_SEEDS = {
     "gqa_causal": 1003,
     "sliding_window": 1004,
     "decode": 1005,
+    "chunked_prefill": 1006,
 }
 
 
@@ -160,6 +165,11 @@ def named(name: str, seed: Optional[int] = None, scale: float = 1.0) -> Workload
     if name == "decode":
         Lk = shrink(_uniform_lengths(rng, 128, 1024, 32768))
         return Workload(name, [1] * 128, Lk, 32, 8, 128, False, 0, s)
+    if name == "chunked_prefill":
+        Lq = _uniform_lengths(rng, 32, 128, 1024)
+        prefix = _uniform_lengths(rng, 32, 0, 8192)
+        Lq_s, pre_s = shrink(Lq), [int(round(x * scale)) for x in prefix]
+        return Workload(name, Lq_s, [a + b for a, b in zip(Lq_s, pre_s)], 32, 8, 128, True, 0, s)
     raise KeyError(name)
 
 
