@@ -45,7 +45,7 @@ def _load():
         lib = ctypes.CDLL(build())
         fn = lib.oracle_varlen_attention_rows
         fn.restype = ctypes.c_int
-        fn.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6 + [
+        fn.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 6 + [
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
         _lib = lib
@@ -69,11 +69,15 @@ def default_threads() -> int:
 
 def attention_rows(q, k, v, cu_q: Sequence[int], cu_k: Sequence[int], H: int, H_kv: int,
                    D: int, causal: bool, window: int = 0,
-                   rows: Optional[np.ndarray] = None, nthreads: Optional[int] = None):
+                   rows: Optional[np.ndarray] = None, nthreads: Optional[int] = None,
+                   seqused_k: Optional[Sequence[int]] = None):
     """fp64 output rows and logsumexp.
 
     q: [total_q, H, D] bf16; k, v: [total_k, H_kv, D] bf16 (torch bf16 or uint16 bits).
     rows: optional int array [n, 2] of (token, head) pairs; None = all rows.
+    seqused_k: optional per-sequence key counts for a cache with a capacity
+    stride (keys of sequence b: the first min(seqused_k[b], cu_k[b+1] - cu_k[b])
+    rows from cu_k[b]); None = every row of the sequence's range.
     Returns (out [n, D] float64, lse [n] float64); with rows=None, shaped
     [total_q, H, D] and [total_q, H].
     """
@@ -82,6 +86,12 @@ def attention_rows(q, k, v, cu_q: Sequence[int], cu_k: Sequence[int], H: int, H_
     cq = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int32))
     ck = np.ascontiguousarray(np.asarray(cu_k, dtype=np.int32))
     batch = len(cq) - 1
+    used_p = None
+    if seqused_k is not None:
+        used = np.ascontiguousarray(np.asarray(seqused_k, dtype=np.int32))
+        if used.shape != (batch,):
+            raise ValueError("seqused_k must hold one count per sequence")
+        used_p = used.ctypes.data
     total_q = int(cq[-1])
     if rows is None:
         n = total_q * H
@@ -95,7 +105,7 @@ def attention_rows(q, k, v, cu_q: Sequence[int], cu_k: Sequence[int], H: int, H_
     out = np.zeros((n, D), dtype=np.float64)
     lse = np.zeros((n,), dtype=np.float64)
     rc = lib.oracle_varlen_attention_rows(
-        qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, cq.ctypes.data, ck.ctypes.data,
+        qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, cq.ctypes.data, ck.ctypes.data, used_p,
         batch, H, H_kv, D, int(bool(causal)), int(window), tok_p, head_p, n,
         out.ctypes.data, lse.ctypes.data, int(nthreads or default_threads()))
     if rc != 0:

@@ -28,7 +28,13 @@
  *     even without the causal flag;
  *   - logsumexp is the natural log of sum_j exp(s_ij) over the visible keys
  *     of the SCALED scores s_ij = q_i.k_j / sqrt(D);
- *   - a query with no visible key gets output 0 and logsumexp -inf.
+ *   - a query with no visible key gets output 0 and logsumexp -inf;
+ *   - a key-value cache with a capacity stride (the kv_seq_len of flash.rs
+ *     FlashAttentionOps: iterate over the first n positions while the
+ *     tensor's size stays the memory stride), in the packed layout: when
+ *     seqused_k is given, sequence b's key rows still start at cu_k[b] but
+ *     only the first min(seqused_k[b], cu_k[b+1] - cu_k[b]) are its keys,
+ *     and that count is the L_k of every rule above.
  *
  * Inputs are bf16 bit patterns; each is widened exactly to double.  All
  * arithmetic is double.  Rows are independent, so threads split the list of
@@ -74,6 +80,7 @@ static int key_visible(int64_t i, int64_t j, int64_t L_q, int64_t L_k,
 typedef struct {
     const uint16_t *q, *k, *v;
     const int32_t *cu_q, *cu_k;
+    const int32_t* seqused_k; /* NULL => every row of the sequence's range is a key */
     int batch, H, H_kv, D, causal, window;
     const int64_t* row_token; /* NULL => all rows r = t*H + h */
     const int32_t* row_head;
@@ -91,7 +98,11 @@ static void one_row(const job_t* jb, int64_t r, double* s) {
     const int D = jb->D;
     const int b = owning_sequence(jb->cu_q, jb->batch, t);
     const int64_t L_q = (int64_t)jb->cu_q[b + 1] - jb->cu_q[b];
-    const int64_t L_k = (int64_t)jb->cu_k[b + 1] - jb->cu_k[b];
+    int64_t L_k = (int64_t)jb->cu_k[b + 1] - jb->cu_k[b];
+    if (jb->seqused_k) {
+        const int64_t used = jb->seqused_k[b] > 0 ? jb->seqused_k[b] : 0;
+        if (used < L_k) L_k = used;
+    }
     const int64_t i = t - jb->cu_q[b];
     const int group = jb->H / jb->H_kv;
     const int hk = h / group;
@@ -140,6 +151,9 @@ static void* run_job(void* arg) {
  *
  * q, k, v:     bf16 bit patterns, packed [total_q, H, D] and [total_k, H_kv, D].
  * cu_q, cu_k:  host int32 [batch + 1] cumulative lengths.
+ * seqused_k:   optional host int32 [batch]: sequence b's keys are the first
+ *              min(seqused_k[b], cu_k[b+1] - cu_k[b]) rows from cu_k[b]
+ *              (NULL: all of them).
  * row_token, row_head: optional (token, head) pairs to compute (n_rows of
  *              them); when row_token is NULL every row is computed in the
  *              order r = token * H + head and n_rows must be total_q * H.
@@ -147,7 +161,8 @@ static void* run_job(void* arg) {
  * Returns 0, or -1 on an argument error, -2 on an allocation failure.
  */
 int oracle_varlen_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                 const int32_t* cu_q, const int32_t* cu_k, int batch,
+                                 const int32_t* cu_q, const int32_t* cu_k,
+                                 const int32_t* seqused_k, int batch,
                                  int H, int H_kv, int D, int causal, int window,
                                  const int64_t* row_token, const int32_t* row_head,
                                  int64_t n_rows, double* out, double* lse, int nthreads) {
@@ -170,6 +185,7 @@ int oracle_varlen_attention_rows(const uint16_t* q, const uint16_t* k, const uin
     for (int w = 0; w < nthreads; ++w) {
         job_t* jb = &jobs[w];
         jb->q = q; jb->k = k; jb->v = v; jb->cu_q = cu_q; jb->cu_k = cu_k;
+        jb->seqused_k = seqused_k;
         jb->batch = batch; jb->H = H; jb->H_kv = H_kv; jb->D = D;
         jb->causal = causal; jb->window = window;
         jb->row_token = row_token; jb->row_head = row_head;

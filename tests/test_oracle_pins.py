@@ -296,3 +296,48 @@ def test_schedule_key_ranges_match_band_mask(Lq, Lk, causal, W):
     for a, b in zip(items, items[1:]):
         if a[3] - a[2] == b[3] - b[2]:
             assert (a[0], a[1]) < (b[0], b[1])
+
+
+# --- key-value cache with a capacity stride ------------------------------------
+
+@pytest.mark.parametrize("causal,window,H,H_kv", [(False, 0, 4, 2), (True, 0, 2, 1), (True, 5, 4, 4)])
+def test_capacity_stride_equals_compacted_layout(oracle_lib, causal, window, H, H_kv):
+    # flash.rs FlashAttentionOps "kv_seq_len": iterate over the first n key
+    # positions while the buffer's size stays the stride.  In the packed
+    # layout: keys of sequence b are the first min(seqused_k[b], capacity)
+    # rows of its slot.  The same rows copied into a compact packed tensor
+    # (no seqused) must give bitwise the same result: the oracle then sums the
+    # same products in the same order.  Unused slot rows hold large finite
+    # garbage that would change every result if it were read.
+    D = 16
+    L_q = [3, 1, 4, 2, 5]
+    cap = [8, 6, 4, 9, 7]
+    used = [5, 6, 0, 12, 7]  # full slot, empty, beyond the capacity (clamped)
+    cu_q = workloads.cu_seqlens(L_q)
+    cu_cache = workloads.cu_seqlens(cap)
+    g = torch.Generator().manual_seed(11)
+    q = torch.randn(cu_q[-1], H, D, generator=g).to(torch.bfloat16)
+    kc = (torch.randn(cu_cache[-1], H_kv, D, generator=g) * 50).to(torch.bfloat16)
+    vc = (torch.randn(cu_cache[-1], H_kv, D, generator=g) * 50).to(torch.bfloat16)
+    eff = [min(u, c) for u, c in zip(used, cap)]
+    keep = torch.cat([torch.arange(cu_cache[b], cu_cache[b] + eff[b]) for b in range(len(cap))])
+    for b in range(len(cap)):  # the used rows: ordinary N(0, 1) data
+        kc[cu_cache[b]:cu_cache[b] + eff[b]] = torch.randn(eff[b], H_kv, D, generator=g).to(torch.bfloat16)
+        vc[cu_cache[b]:cu_cache[b] + eff[b]] = torch.randn(eff[b], H_kv, D, generator=g).to(torch.bfloat16)
+    o1, l1 = oracle_lib.attention_rows(q, kc, vc, cu_q, cu_cache, H, H_kv, D, causal, window,
+                                       seqused_k=used)
+    o2, l2 = oracle_lib.attention_rows(q, kc[keep], vc[keep], cu_q, workloads.cu_seqlens(eff), H,
+                                       H_kv, D, causal, window)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    # the empty sequence: no visible key
+    b = 2
+    assert np.all(np.isneginf(l1[cu_q[b]:cu_q[b + 1]])) and np.all(o1[cu_q[b]:cu_q[b + 1]] == 0)
+
+
+def test_capacity_stride_with_full_counts_is_the_plain_layout(oracle_lib):
+    wl = workloads.custom([5, 7], [9, 7], 2, 1, 16, True, 0, seed=13)
+    q, k, v = workloads.make_qkv(wl)
+    o1, l1 = _run(oracle_lib, wl, q, k, v)
+    o2, l2 = oracle_lib.attention_rows(q, k, v, wl.cu_q, wl.cu_k, wl.H, wl.H_kv, wl.D, wl.causal,
+                                       wl.window, seqused_k=wl.lengths_k)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
