@@ -81,6 +81,28 @@ int varlen_attention_fwd(const void* q, const void* k, const void* v,
                          int causal, int window, void* out, float* lse, void* stream);
 
 /*
+ * varlen_attention_fwd over a key-value cache with a capacity stride: the
+ * packed form of the kv_seq_len argument of boostr flash.rs FlashAttentionOps
+ * (section "kv_seq_len": iterate over the first n key positions while the
+ * buffer's size stays the memory stride, so a full-capacity cache is passed
+ * without copying).  Sequence b's slot is key/value rows cu_seqlens_k[b] ..
+ * cu_seqlens_k[b+1]-1; its keys are the first min(seqused_k[b], slot size)
+ * of them, and that count is the key length of the causal (bottom-right),
+ * window and empty-row rules.  seqused_k is device int32 [batch], required
+ * (VA_ERR_INVALID_ARG when NULL).  Slot rows past a sequence's count are
+ * never visible but may be read and multiplied by exact zeros, so they must
+ * hold finite values (zeros or stale keys, not NaN/inf).  max_seqlen_k bounds
+ * the slot sizes.  Everything else as for varlen_attention_fwd (decode path
+ * when max_seqlen_q == 1).
+ */
+int varlen_attention_fwd_kvcache(const void* q, const void* k, const void* v,
+                                 const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                 const int32_t* seqused_k, int batch, int num_heads,
+                                 int num_kv_heads, int max_seqlen_q, int max_seqlen_k,
+                                 int head_dim, int causal, int window, void* out, float* lse,
+                                 void* stream);
+
+/*
  * Same as varlen_attention_fwd with the path forced (VA_PATH_*) and, for the
  * decode path, the number of keys per split (decode_split_keys in [32, 65536];
  * 0 = library default: the largest of 4096, 2048, ..., 256 keys that still

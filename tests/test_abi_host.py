@@ -75,3 +75,10 @@ def test_decode_split_keys_range_checked(lib):
     assert rc == -1 and "path" in lib.varlen_attention_last_error().decode()
     rc = f(16, 16, 16, 16, 16, 1, 4, 2, 8, 8, 64, 0, 0, 16, 16, 2, 0, None)
     assert rc == -1 and "max_seqlen_q" in lib.varlen_attention_last_error().decode()
+
+
+def test_kvcache_entry_requires_seqused_without_gpu(lib):
+    rc = lib.varlen_attention_fwd_kvcache(16, 16, 16, 16, 16, None, 1, 4, 2, 8, 8, 64, 1, 0, 16, 16,
+                                          None)
+    assert rc == -1
+    assert b"seqused_k is NULL" in lib.varlen_attention_last_error()

@@ -26,6 +26,7 @@ _P, _I = ctypes.c_void_p, ctypes.c_int
 SIGNATURES = {
     "varlen_attention_fwd": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_fwd_ex": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _I, _I, _P]),
+    "varlen_attention_fwd_kvcache": (_I, [_P, _P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_fwd_host": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_schedule": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P]),
@@ -119,6 +120,36 @@ def varlen_attention_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         rc = lib.varlen_attention_fwd_ex(*args, int(path), int(decode_split_keys),
                                          _stream_ptr(stream))
     _check(rc)
+    return out, lse
+
+
+def varlen_attention_fwd_kvcache(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                 cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                                 seqused_k: torch.Tensor, batch: int, num_heads: int,
+                                 num_kv_heads: int, max_seqlen_q: int, max_seqlen_k: int,
+                                 head_dim: int, causal: bool, window: int = 0,
+                                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                                 stream: Optional[torch.cuda.Stream] = None
+                                 ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Attention over a capacity-strided key-value cache: sequence b's keys are the
+    first seqused_k[b] rows of its slot cu_seqlens_k[b]..cu_seqlens_k[b+1]-1."""
+    lib = load()
+    _check_inputs(q, k, v, cu_seqlens_q, cu_seqlens_k, num_heads, num_kv_heads, head_dim, "cuda")
+    if (seqused_k.dtype != torch.int32 or not seqused_k.is_contiguous()
+            or seqused_k.device.type != "cuda" or seqused_k.shape != (batch,)):
+        raise ValueError("seqused_k must be a contiguous int32 cuda tensor of shape [batch]")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[0], num_heads, dtype=torch.float32, device=q.device)
+    if out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q")
+    if lse.shape != (q.shape[0], num_heads) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [total_q, num_heads] tensor")
+    _check(lib.varlen_attention_fwd_kvcache(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(),
+        seqused_k.data_ptr(), batch, num_heads, num_kv_heads, max_seqlen_q, max_seqlen_k, head_dim,
+        int(bool(causal)), int(window), out.data_ptr(), lse.data_ptr(), _stream_ptr(stream)))
     return out, lse
 
 

@@ -45,6 +45,7 @@ constexpr float kDecodeRescaleThreshold = 8.0f;
 struct DecodeParams {
     const int* cu_q;
     const int* cu_k;
+    const int* seqused_k;  // optional key counts of a capacity-strided cache (else NULL)
     int batch, H, H_kv, causal, window;
     const __nv_bfloat16* q;
     const __nv_bfloat16* k;
@@ -83,7 +84,7 @@ struct DecodeSmem {
 __device__ __forceinline__ void decode_row_interval(const DecodeParams& p, int b, int& L_q,
                                                    int& lo, int& hi) {
     L_q = p.cu_q[b + 1] - p.cu_q[b];
-    const int L_k = p.cu_k[b + 1] - p.cu_k[b];
+    const int L_k = seq_key_count(p.cu_k, p.seqused_k, b);
     row_key_interval(0, L_q, L_k, p.causal != 0, p.window, lo, hi);
 }
 

@@ -46,6 +46,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow to 2^8 befo
 struct PrefillParams {
     const int* cu_q;
     const int* cu_k;
+    const int* seqused_k;  // optional key counts of a capacity-strided cache (else NULL)
     int batch, H, H_kv, causal, window;
     const TileEntry* tiles;
     SchedHeader* hdr;
@@ -102,7 +103,7 @@ __device__ __forceinline__ void decode_item(const PrefillParams& p, int idx, int
     it.hi = te.kt_hi;
     const int cq = p.cu_q[it.b], ck = p.cu_k[it.b];
     it.L_q = p.cu_q[it.b + 1] - cq;
-    it.L_k = p.cu_k[it.b + 1] - ck;
+    it.L_k = seq_key_count(p.cu_k, p.seqused_k, it.b);
     it.q_row0 = cq + it.qb * kBlockQ;
     it.k_row0 = ck;
 #pragma unroll

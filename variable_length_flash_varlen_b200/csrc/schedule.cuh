@@ -42,6 +42,17 @@ __host__ __device__ __forceinline__ void row_key_interval(int i, int L_q, int L_
     }
 }
 
+// Keys of sequence b: its rows cu_k[b]..cu_k[b+1]-1, or, for a key-value cache
+// with a capacity stride (flash.rs FlashAttentionOps docs, "kv_seq_len": iterate
+// over the first n positions while the buffer size stays the stride), only the
+// first seqused_k[b] of them (clamped to that range) when seqused_k is given.
+__host__ __device__ __forceinline__ int seq_key_count(const int* cu_k, const int* seqused_k, int b) {
+    const int cap = cu_k[b + 1] - cu_k[b];
+    if (!seqused_k) return cap;
+    const int used = seqused_k[b] > 0 ? seqused_k[b] : 0;
+    return used < cap ? used : cap;
+}
+
 // Key-tile range of query rows [first, first + rows) clipped to L_q.  The
 // intervals of consecutive rows have non-decreasing ends and overlap or
 // touch, so the union over the rows is the interval of the first non-empty

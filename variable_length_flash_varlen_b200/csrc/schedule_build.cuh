@@ -46,7 +46,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* red, int& total)
 // scratch: [capacity] enumeration-ordered entries; out: [capacity] sorted.
 // Dynamic shared memory: 8 bytes per key slot (a power of two <= kSortCapacity).
 __global__ void __launch_bounds__(kBuildThreads, 1)
-build_schedule_kernel(const int* __restrict__ cu_q, const int* __restrict__ cu_k, int batch,
+build_schedule_kernel(const int* __restrict__ cu_q, const int* __restrict__ cu_k,
+                      const int* __restrict__ seqused_k, int batch,
                       int causal, int window, int capacity, int key_slots,
                       TileEntry* __restrict__ scratch, TileEntry* __restrict__ out,
                       SchedHeader* __restrict__ hdr) {
@@ -76,7 +77,7 @@ build_schedule_kernel(const int* __restrict__ cu_q, const int* __restrict__ cu_k
         int n = 0, Lq = 0, Lk = 0;
         if (b < batch) {
             Lq = cu_q[b + 1] - cu_q[b];
-            Lk = cu_k[b + 1] - cu_k[b];
+            Lk = seq_key_count(cu_k, seqused_k, b);
             n = (Lq + kBlockQ - 1) / kBlockQ;
         }
         int chunk_total;

@@ -156,6 +156,7 @@ struct Args {
     int batch, H, H_kv, max_q, max_k, D, causal, window;
     void* out;
     float* lse;
+    const int32_t* seqused_k = nullptr;  // key counts of a capacity-strided cache, or NULL
 };
 
 int validate(const Args& a) {
@@ -213,7 +214,7 @@ int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
     }
 
     va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
-        a.cu_q, a.cu_k, a.batch, a.causal, a.window, cap, key_slots, scratch, tiles, hdr);
+        a.cu_q, a.cu_k, a.seqused_k, a.batch, a.causal, a.window, cap, key_slots, scratch, tiles, hdr);
     cudaError_t be = cudaGetLastError();
     if (be != cudaSuccess) {
         cudaFreeAsync(ws, stream);
@@ -223,6 +224,7 @@ int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
     va::PrefillParams p;
     p.cu_q = a.cu_q;
     p.cu_k = a.cu_k;
+    p.seqused_k = a.seqused_k;
     p.batch = a.batch;
     p.H = a.H;
     p.H_kv = a.H_kv;
@@ -288,6 +290,7 @@ int run_decode(const Args& a, const DeviceInfo& dev, int split_keys, cudaStream_
     va::DecodeParams p;
     p.cu_q = a.cu_q;
     p.cu_k = a.cu_k;
+    p.seqused_k = a.seqused_k;
     p.batch = a.batch;
     p.H = a.H;
     p.H_kv = a.H_kv;
@@ -436,13 +439,14 @@ int run_prefill_noalloc(const Args& a, cudaStream_t stream) {
     // the builder rewrites the whole header (count and work counter) and every
     // list entry it hands out, so nothing left by the previous call is read
     va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
-        a.cu_q, a.cu_k, a.batch, a.causal, a.window, cap, key_slots, scratch, tiles, hdr);
+        a.cu_q, a.cu_k, a.seqused_k, a.batch, a.causal, a.window, cap, key_slots, scratch, tiles, hdr);
     cudaError_t be = cudaGetLastError();
     if (be != cudaSuccess) return cuda_fail(be, "schedule build launch");
 
     va::PrefillParams p;
     p.cu_q = a.cu_q;
     p.cu_k = a.cu_k;
+    p.seqused_k = a.seqused_k;
     p.batch = a.batch;
     p.H = a.H;
     p.H_kv = a.H_kv;
@@ -478,6 +482,19 @@ int varlen_attention_fwd(const void* q, const void* k, const void* v, const int3
     g_last_error[0] = 0;
     Args a{q, k, v, cu_seqlens_q, cu_seqlens_k, batch, num_heads, num_kv_heads, max_seqlen_q,
            max_seqlen_k, head_dim, causal ? 1 : 0, window, out, lse};
+    return forward(a, VA_PATH_AUTO, 0, static_cast<cudaStream_t>(stream));
+}
+
+int varlen_attention_fwd_kvcache(const void* q, const void* k, const void* v,
+                                 const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                 const int32_t* seqused_k, int batch, int num_heads,
+                                 int num_kv_heads, int max_seqlen_q, int max_seqlen_k, int head_dim,
+                                 int causal, int window, void* out, float* lse, void* stream) {
+    g_last_error[0] = 0;
+    if (!seqused_k) return fail(VA_ERR_INVALID_ARG, "seqused_k is NULL (use varlen_attention_fwd)");
+    Args a{q, k, v, cu_seqlens_q, cu_seqlens_k, batch, num_heads, num_kv_heads, max_seqlen_q,
+           max_seqlen_k, head_dim, causal ? 1 : 0, window, out, lse};
+    a.seqused_k = seqused_k;
     return forward(a, VA_PATH_AUTO, 0, static_cast<cudaStream_t>(stream));
 }
 
@@ -571,7 +588,7 @@ int varlen_attention_schedule(const int32_t* cu_seqlens_q, const int32_t* cu_seq
     VA_CUDA(ws_alloc(reinterpret_cast<void**>(&ws), 256 + list_bytes, stream));
     auto* hdr = reinterpret_cast<va::SchedHeader*>(ws);
     va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
-        cu_seqlens_q, cu_seqlens_k, batch, causal ? 1 : 0, window, capacity, key_slots,
+        cu_seqlens_q, cu_seqlens_k, nullptr, batch, causal ? 1 : 0, window, capacity, key_slots,
         reinterpret_cast<va::TileEntry*>(ws + 256), reinterpret_cast<va::TileEntry*>(tiles), hdr);
     cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess)
