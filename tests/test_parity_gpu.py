@@ -68,6 +68,21 @@ def test_edge_cases_match_oracle(oracle_lib, case):
     compare(out, lse, ref_o, ref_l)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("tail", [1, 5, 8, 9, 63, 64, 120, 127])
+def test_ragged_last_tile_matches_oracle(oracle_lib, tail, D):
+    # the packed tensors end `tail` rows into a 128-row tile: the last query and
+    # key tiles are copied as whole 8-row groups plus one partial group, the
+    # rest of the tile zero (fewer than 8 rows: no whole group at all)
+    L = [256, 128 + tail]
+    for causal in (True, False):
+        wl = workloads.custom(L, L, 4, 2, D, causal, 0, seed=100 + tail)
+        q, k, v = workloads.make_qkv(wl)
+        out, lse = run_gpu(wl, q, k, v, path=binding.VA_PATH_PREFILL)
+        ref_o, ref_l = oracle_all(oracle_lib, wl, q, k, v)
+        compare(out, lse, ref_o, ref_l)
+
+
 def test_large_scores_stay_finite(oracle_lib):
     # scores spanning +-40 in base-e units exercise the reference-max update
     wl = workloads.custom([700, 300], [700, 300], 2, 1, 128, True, 0, seed=5)
@@ -158,6 +173,19 @@ def test_decode_edge_cases(oracle_lib, case):
     for split in (0, 64):
         out, lse = run_gpu(wl, q, k, v, path=binding.VA_PATH_DECODE, split_keys=split)
         compare(out, lse, ref_o, ref_l)
+
+
+@pytest.mark.parametrize("tail", [1, 7, 8, 15, 56, 63])
+def test_decode_ragged_last_tile(oracle_lib, tail):
+    # the packed keys end `tail` rows into a 64-key tile of the decode stream
+    Lk = [640, 320 + tail]
+    for D in (64, 128):
+        wl = workloads.custom([1, 1], Lk, 8, 2, D, False, 0, seed=200 + tail)
+        q, k, v = workloads.make_qkv(wl)
+        ref_o, ref_l = oracle_all(oracle_lib, wl, q, k, v)
+        for split in (0, 64):
+            out, lse = run_gpu(wl, q, k, v, path=binding.VA_PATH_DECODE, split_keys=split)
+            compare(out, lse, ref_o, ref_l)
 
 
 def test_decode_large_scores(oracle_lib):

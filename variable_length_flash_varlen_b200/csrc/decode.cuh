@@ -12,7 +12,7 @@
 // warp instead of ~45 scalar ones (rows past the group's head count are zero
 // and discarded).  Persistent CTAs (one per SM) claim units from a counter.
 // Per CTA: warp 4 streams 64-key tiles of K and V (TMA, 128-byte swizzle;
-// plain loads for a tile that runs past the end of the packed tensor) into a
+// 8-row boxes and plain loads for a tile that runs past the end of the packed tensor) into a
 // ring; warps 0-3 each take 16 keys of every tile and keep, per head, a
 // running max m (base-2 scaled scores, moved lazily by more than 2^8), a
 // running sum l and an unnormalised output.  At the end of a unit the four
@@ -115,6 +115,7 @@ __device__ __forceinline__ bool decode_unit(const DecodeParams& p, int u, Decode
 template <int D>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
 decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ CUtensorMap tmK8, const __grid_constant__ CUtensorMap tmV8,
                      const DecodeParams p) {
     using L = DecodeSmem<D>;
     constexpr int S = L::kStages;
@@ -200,23 +201,60 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                     }
                     __syncwarp();
                 } else {
-                    // the same swizzled layout, rows at or past T_k zero
+                    // The same swizzled layout, rows at or past T_k zero: whole 8-row
+                    // groups before T_k by TMA in 8-row boxes (a box written at a
+                    // 1024-byte-aligned offset has the swizzle phase of those rows of a
+                    // full box), the one partial group by plain loads all in flight at
+                    // once, the rest zero-filled.  (The maps' row extent is only an
+                    // upper bound of T_k, so no box may reach past it.)
                     constexpr int kVecPerRow = D / 8;
-                    for (int idx = lane; idx < kDecodeTileKeys * kVecPerRow; idx += 32) {
-                        const int r = idx / kVecPerRow, c = idx % kVecPerRow;
-                        uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
-                        if (row0 + r < T_k) {
+                    constexpr int kTailPerLane = 8 * kVecPerRow / 32;
+                    const int valid = max(0, min(kDecodeTileKeys, T_k - row0));
+                    const int g8 = valid >> 3, tail0 = g8 << 3;
+                    auto swz = [](int r, int c) {
+                        return (c >> 3) * L::kHalfBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+                    };
+                    uint4 kvals[kTailPerLane], vvals[kTailPerLane];
+#pragma unroll
+                    for (int u = 0; u < kTailPerLane; ++u) {
+                        const int idx = lane + 32 * u;
+                        const int r = tail0 + idx / kVecPerRow, c = idx % kVecPerRow;
+                        kvals[u] = make_uint4(0u, 0u, 0u, 0u);
+                        vvals[u] = kvals[u];
+                        if (r < valid) {
                             const size_t off = static_cast<size_t>(row0 + r) * stride + w.hk * D + c * 8;
-                            kv = *reinterpret_cast<const uint4*>(p.k + off);
-                            vv = *reinterpret_cast<const uint4*>(p.v + off);
+                            kvals[u] = *reinterpret_cast<const uint4*>(p.k + off);
+                            vvals[u] = *reinterpret_cast<const uint4*>(p.v + off);
                         }
-                        const int dst = (c >> 3) * L::kHalfBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-                        *reinterpret_cast<uint4*>(kt + dst) = kv;
-                        *reinterpret_cast<uint4*>(vt + dst) = vv;
+                    }
+#pragma unroll
+                    for (int u = 0; u < kTailPerLane; ++u) {
+                        const int idx = lane + 32 * u;
+                        const int r = tail0 + idx / kVecPerRow, c = idx % kVecPerRow;
+                        if (r < kDecodeTileKeys) {
+                            *reinterpret_cast<uint4*>(kt + swz(r, c)) = kvals[u];
+                            *reinterpret_cast<uint4*>(vt + swz(r, c)) = vvals[u];
+                        }
+                    }
+                    for (int idx = lane; idx < (kDecodeTileKeys - tail0 - 8) * kVecPerRow; idx += 32) {
+                        const int r = tail0 + 8 + idx / kVecPerRow, c = idx % kVecPerRow;
+                        *reinterpret_cast<uint4*>(kt + swz(r, c)) = make_uint4(0u, 0u, 0u, 0u);
+                        *reinterpret_cast<uint4*>(vt + swz(r, c)) = make_uint4(0u, 0u, 0u, 0u);
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&full[s]);
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(2 * g8 * (D / 64) * 1024));
+                        for (int g = 0; g < g8; ++g) {
+#pragma unroll
+                            for (int h = 0; h < D / 64; ++h) {
+                                tma_load_2d(kt + h * L::kHalfBytes + g * 1024, &tmK8, w.hk * D + h * 64,
+                                            row0 + g * 8, &full[s]);
+                                tma_load_2d(vt + h * L::kHalfBytes + g * 1024, &tmV8, w.hk * D + h * 64,
+                                            row0 + g * 8, &full[s]);
+                            }
+                        }
+                    }
                     __syncwarp();
                 }
             }

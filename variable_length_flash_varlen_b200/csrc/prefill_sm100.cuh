@@ -14,8 +14,8 @@
 //               one half's MMAs run while the other half's softmax does
 //   warp 9      producer: claims work items from a grid-wide counter (longest
 //               first), TMA tile loads of Q, K, V into 128-byte-swizzled
-//               shared memory (plain loads for a tile that runs past the end
-//               of the packed tensor)
+//               shared memory (8-row boxes and one group of plain loads for
+//               a tile that runs past the end of the packed tensor)
 // Tensor memory (512 columns): S_0 at 0, S_1 at 128 (P_h aliases the first
 // 64 columns of S_h), O_0 at 256, O_1 at 256 + D.
 //
@@ -116,30 +116,74 @@ __device__ __forceinline__ bool takes_part(const Item& it, int x, int kt) {
     return it.lo_h[x] <= kt && kt < it.hi_h[x];
 }
 
-// Copy a 128-row tile whose rows may run past `T` with plain loads, writing
-// the 128-byte-swizzle layout TMA would have produced; rows >= T become zero.
+// Tensor maps of the three inputs, each as a 2-D view [rows][heads * D] with
+// 64-column boxes and 128-byte swizzle: one with 128-row boxes for whole
+// tiles and one with 8-row boxes (one swizzle atom high) for a tile that runs
+// past the end of the packed tensor.  The row extent of every map is only an
+// upper bound of the packed length (batch * max_seqlen; the exact total lives
+// in cu_seqlens on the device), so no box may cover a row at or past it.
+struct PrefillMaps {
+    CUtensorMap q, k, v;     // 128-row boxes
+    CUtensorMap q8, k8, v8;  // 8-row boxes
+};
+
+// A 128-row tile whose rows run past the packed length `T`, in the
+// 128-byte-swizzle layout a full-tile copy would produce, rows >= T zero.
+// The whole groups of 8 rows before T come by TMA in 8-row boxes (a box
+// written at a 1024-byte-aligned offset carries the same swizzle phase as
+// those rows of a full box); the one partial group is read with plain loads,
+// all in flight at once, and the rows after it are zero-filled.  Completion is
+// signalled on `full` (one arrival, carrying the TMA byte count).
 template <int D>
-__device__ __forceinline__ void load_tile_plain(uint8_t* dst, const __nv_bfloat16* src, int row0,
-                                                int T, int row_stride, int col0, int lane) {
-    constexpr int kVecPerRow = D / 8;  // 16-byte vectors per row
-    for (int idx = lane; idx < 128 * kVecPerRow; idx += 32) {
-        const int r = idx / kVecPerRow, c = idx % kVecPerRow;
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (row0 + r < T) {
-            val = *reinterpret_cast<const uint4*>(src + static_cast<size_t>(row0 + r) * row_stride +
-                                                  col0 + c * 8);
-        }
-        const int sub = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4*>(dst + sub * PrefillSmem<D>::kChunkBytes + r * 128 +
-                                  ((cc ^ (r & 7)) << 4)) = val;
+__device__ __forceinline__ void load_tile_ragged(uint8_t* dst, const CUtensorMap* map8,
+                                                 const __nv_bfloat16* src, int row0, int T,
+                                                 int row_stride, int col0, uint64_t* full, int lane) {
+    constexpr int kVecPerRow = D / 8;                 // 16-byte vectors per row
+    constexpr int kTailVec = 8 * kVecPerRow;          // one 8-row group
+    constexpr int kTailPerLane = kTailVec / 32;
+    const int valid = max(0, min(128, T - row0));    // rows before T (< 128 here)
+    const int g8 = valid >> 3;                        // whole 8-row groups by TMA
+    const int tail0 = g8 << 3;                        // first row of the partial group
+    auto swz = [&](int r, int c) {
+        return dst + (c >> 3) * PrefillSmem<D>::kChunkBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+    };
+    uint4 vals[kTailPerLane];
+#pragma unroll
+    for (int u = 0; u < kTailPerLane; ++u) {
+        const int idx = lane + 32 * u;
+        const int r = tail0 + idx / kVecPerRow, c = idx % kVecPerRow;
+        vals[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (r < valid)
+            vals[u] = *reinterpret_cast<const uint4*>(src + static_cast<size_t>(row0 + r) * row_stride +
+                                                      col0 + c * 8);
+    }
+#pragma unroll
+    for (int u = 0; u < kTailPerLane; ++u) {
+        const int idx = lane + 32 * u;
+        const int r = tail0 + idx / kVecPerRow, c = idx % kVecPerRow;
+        if (r < 128) *reinterpret_cast<uint4*>(swz(r, c)) = vals[u];
+    }
+    for (int idx = lane; idx < (128 - tail0 - 8) * kVecPerRow; idx += 32) {
+        const int r = tail0 + 8 + idx / kVecPerRow, c = idx % kVecPerRow;
+        *reinterpret_cast<uint4*>(swz(r, c)) = make_uint4(0u, 0u, 0u, 0u);
     }
     fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        mbar_arrive_expect_tx(full, static_cast<uint32_t>(g8 * PrefillSmem<D>::kChunks * 1024));
+        for (int g = 0; g < g8; ++g) {
+#pragma unroll
+            for (int c = 0; c < PrefillSmem<D>::kChunks; ++c)
+                tma_load_2d(dst + c * PrefillSmem<D>::kChunkBytes + g * 1024, map8, col0 + c * 64,
+                            row0 + g * 8, full);
+        }
+    }
     __syncwarp();
 }
 
 // Whole warp: one 128-row tile into `dst`, completion signalled on `full`.
 template <int D>
-__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map,
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, const CUtensorMap* map8,
                                           const __nv_bfloat16* src, int row0, int T, int row_stride,
                                           int col0, uint64_t* full, int lane) {
     if (row0 + 128 <= T) {
@@ -151,9 +195,7 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map,
         }
         __syncwarp();
     } else {
-        load_tile_plain<D>(dst, src, row0, T, row_stride, col0, lane);
-        if (lane == 0) mbar_arrive(full);
-        __syncwarp();
+        load_tile_ragged<D>(dst, map8, src, row0, T, row_stride, col0, full, lane);
     }
 }
 
@@ -167,8 +209,7 @@ __device__ __forceinline__ void store_row_zero(const PrefillParams& p, size_t ou
 
 template <int D>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
-prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams p) {
     using L = PrefillSmem<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -220,9 +261,9 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         tmem_relinquish();
     }
     if (warp == kLoadWarp && lane == 0) {
-        prefetch_tensormap(&tmQ);
-        prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmV);
+        prefetch_tensormap(&maps.q);
+        prefetch_tensormap(&maps.k);
+        prefetch_tensormap(&maps.v);
     }
     tc_fence_before();
     __syncthreads();
@@ -265,7 +306,7 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
                 if (it.hi_h[x] > it.lo_h[x]) {
-                    load_tile<D>(smem + L::kQ + x * L::kTileBytes, &tmQ, p.q, it.q_row0 + x * kBlockM,
+                    load_tile<D>(smem + L::kQ + x * L::kTileBytes, &maps.q, &maps.q8, p.q, it.q_row0 + x * kBlockM,
                                  T_q, q_stride, it.h * D, &q_full[x], lane);
                     ++q_issued[x];
                 }
@@ -274,11 +315,11 @@ prefill_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 const int s = k_issued % kStages;
                 const uint32_t ph = (k_issued / kStages) & 1;
                 if (!(ok = mbar_wait_warp(&k_empty[s], ph ^ 1, abort_flag, status))) break;
-                load_tile<D>(smem + L::kK + s * L::kTileBytes, &tmK, p.k, it.k_row0 + kt * kBlockN,
+                load_tile<D>(smem + L::kK + s * L::kTileBytes, &maps.k, &maps.k8, p.k, it.k_row0 + kt * kBlockN,
                              T_k, kv_stride, it.hk * D, &k_full[s], lane);
                 ++k_issued;
                 if (!(ok = mbar_wait_warp(&v_empty[s], ph ^ 1, abort_flag, status))) break;
-                load_tile<D>(smem + L::kV + s * L::kTileBytes, &tmV, p.v, it.k_row0 + kt * kBlockN,
+                load_tile<D>(smem + L::kV + s * L::kTileBytes, &maps.v, &maps.v8, p.v, it.k_row0 + kt * kBlockN,
                              T_k, kv_stride, it.hk * D, &v_full[s], lane);
                 ++v_issued;
             }

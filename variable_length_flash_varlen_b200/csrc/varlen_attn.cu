@@ -186,6 +186,24 @@ int validate(const Args& a) {
     return VA_OK;
 }
 
+// Tensor maps of the prefill kernel: Q, K, V as [rows][heads * D] with an
+// upper-bound row extent (batch * max_seqlen), 128-row and 8-row boxes.
+int make_prefill_maps(const Args& a, va::PrefillMaps* m) {
+    const long long rows_q = std::max(1ll, static_cast<long long>(a.batch) * a.max_q);
+    const long long rows_k = std::max(1ll, static_cast<long long>(a.batch) * a.max_k);
+    const long long cols_q = static_cast<long long>(a.H) * a.D;
+    const long long cols_k = static_cast<long long>(a.H_kv) * a.D;
+    int rc;
+    if ((rc = make_tile_map(&m->q, a.q, cols_q, rows_q, va::kBlockM)) != VA_OK ||
+        (rc = make_tile_map(&m->k, a.k, cols_k, rows_k, va::kBlockN)) != VA_OK ||
+        (rc = make_tile_map(&m->v, a.v, cols_k, rows_k, va::kBlockN)) != VA_OK ||
+        (rc = make_tile_map(&m->q8, a.q, cols_q, rows_q, 8)) != VA_OK ||
+        (rc = make_tile_map(&m->k8, a.k, cols_k, rows_k, 8)) != VA_OK ||
+        (rc = make_tile_map(&m->v8, a.v, cols_k, rows_k, 8)) != VA_OK)
+        return rc;
+    return VA_OK;
+}
+
 int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
     const long long tiles_per_seq = (a.max_q + va::kBlockQ - 1) / va::kBlockQ;
     const long long cap_ll = tiles_per_seq * a.batch;
@@ -203,12 +221,8 @@ int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
     auto* tiles = reinterpret_cast<va::TileEntry*>(ws + hdr_bytes + list_bytes);
 
     int rc = VA_OK;
-    CUtensorMap tq, tk, tv;
-    const long long rows_q = std::max(1ll, static_cast<long long>(a.batch) * a.max_q);
-    const long long rows_k = std::max(1ll, static_cast<long long>(a.batch) * a.max_k);
-    if ((rc = make_tile_map(&tq, a.q, static_cast<long long>(a.H) * a.D, rows_q, va::kBlockM)) != VA_OK ||
-        (rc = make_tile_map(&tk, a.k, static_cast<long long>(a.H_kv) * a.D, rows_k, va::kBlockN)) != VA_OK ||
-        (rc = make_tile_map(&tv, a.v, static_cast<long long>(a.H_kv) * a.D, rows_k, va::kBlockN)) != VA_OK) {
+    va::PrefillMaps maps;
+    if ((rc = make_prefill_maps(a, &maps)) != VA_OK) {
         cudaFreeAsync(ws, stream);
         return rc;
     }
@@ -242,9 +256,9 @@ int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
     const long long items = cap_ll * a.H;
     const int grid = static_cast<int>(std::min<long long>(dev.num_sms, items));
     if (a.D == 64)
-        va::prefill_fwd_kernel<64><<<grid, va::kPrefillThreads, va::PrefillSmem<64>::kAlloc, stream>>>(tq, tk, tv, p);
+        va::prefill_fwd_kernel<64><<<grid, va::kPrefillThreads, va::PrefillSmem<64>::kAlloc, stream>>>(maps, p);
     else
-        va::prefill_fwd_kernel<128><<<grid, va::kPrefillThreads, va::PrefillSmem<128>::kAlloc, stream>>>(tq, tk, tv, p);
+        va::prefill_fwd_kernel<128><<<grid, va::kPrefillThreads, va::PrefillSmem<128>::kAlloc, stream>>>(maps, p);
     cudaError_t le = cudaGetLastError();
     cudaFreeAsync(ws, stream);
     if (le != cudaSuccess) return cuda_fail(le, "prefill launch");
@@ -278,11 +292,14 @@ int run_decode(const Args& a, const DeviceInfo& dev, int split_keys, cudaStream_
         cudaFreeAsync(ws, stream);
         return cuda_fail(e, "cudaMemsetAsync (decode work counter)");
     }
-    CUtensorMap tk, tv;
+    CUtensorMap tk, tv, tk8, tv8;
     const long long rows_k = std::max(1ll, static_cast<long long>(a.batch) * a.max_k);
+    const long long cols_k = static_cast<long long>(a.H_kv) * a.D;
     int rc;
-    if ((rc = make_tile_map(&tk, a.k, static_cast<long long>(a.H_kv) * a.D, rows_k, va::kDecodeTileKeys)) != VA_OK ||
-        (rc = make_tile_map(&tv, a.v, static_cast<long long>(a.H_kv) * a.D, rows_k, va::kDecodeTileKeys)) != VA_OK) {
+    if ((rc = make_tile_map(&tk, a.k, cols_k, rows_k, va::kDecodeTileKeys)) != VA_OK ||
+        (rc = make_tile_map(&tv, a.v, cols_k, rows_k, va::kDecodeTileKeys)) != VA_OK ||
+        (rc = make_tile_map(&tk8, a.k, cols_k, rows_k, 8)) != VA_OK ||
+        (rc = make_tile_map(&tv8, a.v, cols_k, rows_k, 8)) != VA_OK) {
         cudaFreeAsync(ws, stream);
         return rc;
     }
@@ -310,10 +327,10 @@ int run_decode(const Args& a, const DeviceInfo& dev, int split_keys, cudaStream_
     p.lse = a.lse;
     const int grid = static_cast<int>(std::min<long long>(dev.num_sms, n_units));
     if (a.D == 64) {
-        va::decode_stream_kernel<64><<<grid, va::kDecodeThreads, va::DecodeSmem<64>::kAlloc, stream>>>(tk, tv, p);
+        va::decode_stream_kernel<64><<<grid, va::kDecodeThreads, va::DecodeSmem<64>::kAlloc, stream>>>(tk, tv, tk8, tv8, p);
         va::decode_combine_kernel<64><<<a.batch * a.H, 64, 0, stream>>>(p);
     } else {
-        va::decode_stream_kernel<128><<<grid, va::kDecodeThreads, va::DecodeSmem<128>::kAlloc, stream>>>(tk, tv, p);
+        va::decode_stream_kernel<128><<<grid, va::kDecodeThreads, va::DecodeSmem<128>::kAlloc, stream>>>(tk, tv, tk8, tv8, p);
         va::decode_combine_kernel<128><<<a.batch * a.H, 128, 0, stream>>>(p);
     }
     cudaError_t le = cudaGetLastError();
@@ -429,13 +446,8 @@ int run_prefill_noalloc(const Args& a, cudaStream_t stream) {
     auto* scratch = reinterpret_cast<va::TileEntry*>(st->scratch + kNoAllocHeaderBytes);
     auto* tiles = reinterpret_cast<va::TileEntry*>(st->scratch + kNoAllocHeaderBytes + list_bytes);
 
-    CUtensorMap tq, tk, tv;
-    const long long rows_q = std::max(1ll, static_cast<long long>(a.batch) * a.max_q);
-    const long long rows_k = std::max(1ll, static_cast<long long>(a.batch) * a.max_k);
-    if ((rc = make_tile_map(&tq, a.q, static_cast<long long>(a.H) * a.D, rows_q, va::kBlockM)) != VA_OK ||
-        (rc = make_tile_map(&tk, a.k, static_cast<long long>(a.H_kv) * a.D, rows_k, va::kBlockN)) != VA_OK ||
-        (rc = make_tile_map(&tv, a.v, static_cast<long long>(a.H_kv) * a.D, rows_k, va::kBlockN)) != VA_OK)
-        return rc;
+    va::PrefillMaps maps;
+    if ((rc = make_prefill_maps(a, &maps)) != VA_OK) return rc;
     // the builder rewrites the whole header (count and work counter) and every
     // list entry it hands out, so nothing left by the previous call is read
     va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
@@ -463,9 +475,9 @@ int run_prefill_noalloc(const Args& a, cudaStream_t stream) {
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)));
     const int grid = static_cast<int>(std::min<long long>(st->num_sms, blocks * a.H));
     if (a.D == 64)
-        va::prefill_fwd_kernel<64><<<grid, va::kPrefillThreads, va::PrefillSmem<64>::kAlloc, stream>>>(tq, tk, tv, p);
+        va::prefill_fwd_kernel<64><<<grid, va::kPrefillThreads, va::PrefillSmem<64>::kAlloc, stream>>>(maps, p);
     else
-        va::prefill_fwd_kernel<128><<<grid, va::kPrefillThreads, va::PrefillSmem<128>::kAlloc, stream>>>(tq, tk, tv, p);
+        va::prefill_fwd_kernel<128><<<grid, va::kPrefillThreads, va::PrefillSmem<128>::kAlloc, stream>>>(maps, p);
     cudaError_t le = cudaGetLastError();
     if (le != cudaSuccess) return cuda_fail(le, "prefill launch");
     return VA_OK;
