@@ -5,8 +5,11 @@ Prints ONE JSON line (rank 0).  Metric: prefill TFLOP/s of the varlen forward
 non-causal MHA workload (q = k lengths uniform-int in [64, 2048], H = H_kv =
 16, D = 128), with the decode-shape HBM GB/s (128 sequences of one query,
 k lengths uniform-int in [1024, 32768], H = 32, H_kv = 8, D = 128) reported
-beside it under "decode".  A step is one call of the C ABI on one batch:
-schedule build + prefill kernel (decode: split + combine kernels).
+beside it under "decode", the chunked-prefill workload under
+"chunked_prefill" and the same headline workload in FP8 (E4M3 inputs and
+output with per-tensor scales, varlen_attention_fwd_fp8) under "fp8".  A step
+is one call of the C ABI on one batch: schedule build + prefill kernel
+(decode: split + combine kernels).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload NAME]
@@ -380,6 +383,25 @@ def run_ours(args, world, rank, local):
     c_value = sum_over_ranks(cflops * args.steps, world) / c_max / 1e12
     del dqc, dkc, dvc, outc, lsec, qc, kc, vc
 
+    # ---- FP8 (E4M3) forward on the headline workload (flash_attention_fwd_fp8 semantics)
+    fq, fk, fv, fsc = workloads.make_qkv_fp8(wl)
+    dfq, dfk, dfv = fq.to(dev), fk.to(dev), fv.to(dev)
+    fout = torch.empty_like(dfq)
+    flse = torch.empty(wl.total_q, wl.H, dtype=torch.float32, device=dev)
+
+    def fstep():
+        binding.varlen_attention_fwd_fp8(dfq, dfk, dfv, cq, ck, wl.batch, wl.H, wl.H_kv,
+                                         wl.max_seqlen_q, wl.max_seqlen_k, wl.D, wl.causal,
+                                         wl.window, fsc["q_scale"], fsc["k_scale"], fsc["v_scale"],
+                                         fsc["o_scale"], out=fout, lse=flse)
+
+    f_ms, _ = time_device_steps(fstep, args.steps, args.warmup, flush, world, stream)
+    f_max = max_over_ranks(sum(f_ms) / 1e3, world)
+    f_value = total_flops / f_max / 1e12
+    # E4M3 dense tensor peak: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
+    fp8_peak = peak * 2.0
+    del dfq, dfk, dfv, fout, flse, fq, fk, fv
+
     # ---- end to end through the host-buffer entry point (pinned memory)
     qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
     cqh = torch.tensor(wl.cu_q, dtype=torch.int32)
@@ -437,6 +459,14 @@ def run_ours(args, world, rank, local):
                                          "unit": "TFLOP/s", "frac": c_value / world / peak,
                                          "peak_kind": f"{peak_kind} bf16 burst"},
                             "gpu_launches": 2 * args.steps},
+        "fp8": {"workload": args.workload, "entry": "varlen_attention_fwd_fp8", "dtype": "e4m3",
+                "scales": fsc, "value": f_value, "unit": "TFLOP/s",
+                "ms_per_step": f_max / args.steps * 1e3,
+                "roofline": {"bound": "tensor", "achieved": f_value / world, "peak": fp8_peak,
+                             "unit": "TFLOP/s", "frac": f_value / world / fp8_peak,
+                             "peak_kind": f"{peak_kind} bf16 burst x 2 (nominal e4m3 / bf16 ratio)",
+                             "kernel": "prefill_fwd_kernel<128, E4M3> (+ schedule build, same call)"},
+                "gpu_launches": 2 * args.steps},
         "e2e": {"value": e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,

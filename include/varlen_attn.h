@@ -103,6 +103,32 @@ int varlen_attention_fwd_kvcache(const void* q, const void* k, const void* v,
                                  void* stream);
 
 /*
+ * FP8 variant: the forward pass of FlashAttentionOps::flash_attention_fwd_fp8
+ * (boostr flash.rs: per-tensor dequantization scales q_scale, k_scale,
+ * v_scale take the FP8 inputs to FP32, o_scale takes the FP32 output to FP8,
+ * FP32 accumulation inside) on the packed layout of varlen_attention_fwd.
+ * q, k, v and out hold 8-bit E4M3 values (OCP "E4M3FN": bias 7, no
+ * infinities, largest finite 448), one byte per element in the layouts of
+ * the file comment; the element value is code * scale.  Scores are
+ * (q_scale q).(k_scale k) / sqrt(head_dim); out = E4M3(O * o_scale) with
+ * round-to-nearest-even and saturation at +-448, O the attention output of
+ * the dequantized inputs (o_scale multiplies: the FP32 -> FP8 direction the
+ * trait gives it); lse (f32) is the natural-log logsumexp of those scores.
+ * P is rounded to E4M3 before the tensor-core P V product (its row sum is
+ * taken unrounded).  head_dim must be 128 (VA_ERR_UNSUPPORTED otherwise);
+ * the four scales must be finite and > 0 (VA_ERR_INVALID_ARG).  Every query
+ * length runs on the tensor-core tile kernel.  Memory, asynchrony and errors
+ * as for varlen_attention_fwd.
+ */
+int varlen_attention_fwd_fp8(const void* q, const void* k, const void* v,
+                             const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                             int batch, int num_heads, int num_kv_heads,
+                             int max_seqlen_q, int max_seqlen_k, int head_dim,
+                             int causal, int window, float q_scale, float k_scale,
+                             float v_scale, float o_scale, void* out, float* lse,
+                             void* stream);
+
+/*
  * Same as varlen_attention_fwd with the path forced (VA_PATH_*) and, for the
  * decode path, the number of keys per split (decode_split_keys in [32, 65536];
  * 0 = library default: the largest of 4096, 2048, ..., 256 keys that still

@@ -11,6 +11,12 @@ varlen_attention.rs (VarLenAttentionOps, "Layout contract") computed per
 (standard_single_head_attention / standard_softmax); see its header for the
 readings taken where the pages are silent.
 
+``attention_rows_fp8`` is the same definition for E4M3 inputs with
+per-tensor dequantization scales (boostr flash.rs,
+FlashAttentionOps::flash_attention_fwd_fp8); ``e4m3_decode`` /
+``e4m3_encode`` are the format's definition (round to nearest even,
+saturating at +-448) written out in the same C file.
+
 ``schedule`` (in ``oracle/schedule.py``) is the CPU statement of the tile
 work list the GPU scheduler must reproduce bit-exactly.
 """
@@ -48,6 +54,14 @@ def _load():
         fn.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 6 + [
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        f8 = lib.oracle_varlen_attention_rows_fp8
+        f8.restype = ctypes.c_int
+        f8.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_double] * 3 + [ctypes.c_void_p] * 2 + [
+            ctypes.c_int] * 6 + [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64] + [
+            ctypes.c_void_p] * 3 + [ctypes.c_int]
+        for name in ("oracle_e4m3_decode_array", "oracle_e4m3_encode_array"):
+            getattr(lib, name).restype = None
+            getattr(lib, name).argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64]
         _lib = lib
     return _lib
 
@@ -113,3 +127,73 @@ def attention_rows(q, k, v, cu_q: Sequence[int], cu_k: Sequence[int], H: int, H_
     if rows is None:
         return out.reshape(total_q, H, D), lse.reshape(total_q, H)
     return out, lse
+
+
+def _bytes(x) -> np.ndarray:
+    """E4M3 tensor (torch.float8_e4m3fn or uint8 bits) -> contiguous uint8 numpy array."""
+    if hasattr(x, "dtype") and "float8" in str(getattr(x, "dtype")):
+        import torch
+        x = x.detach().cpu().contiguous().view(torch.uint8).numpy()
+    elif hasattr(x, "dtype") and str(getattr(x, "dtype")) == "torch.uint8":
+        x = x.detach().cpu().contiguous().numpy()
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint8:
+        raise TypeError("E4M3 inputs must be float8_e4m3fn tensors or uint8 bit-pattern arrays")
+    return x
+
+
+def e4m3_decode(bits) -> np.ndarray:
+    """E4M3 bit patterns -> float64 values (NaN for the two NaN codes)."""
+    b = _bytes(bits)
+    out = np.empty(b.shape, dtype=np.float64)
+    _load().oracle_e4m3_decode_array(b.ctypes.data, out.ctypes.data, b.size)
+    return out
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """float64 values -> nearest E4M3 bit patterns (ties to even, saturating at +-448)."""
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    out = np.empty(a.shape, dtype=np.uint8)
+    _load().oracle_e4m3_encode_array(a.ctypes.data, out.ctypes.data, a.size)
+    return out
+
+
+def attention_rows_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float,
+                       cu_q: Sequence[int], cu_k: Sequence[int], H: int, H_kv: int, D: int,
+                       causal: bool, window: int = 0, rows: Optional[np.ndarray] = None,
+                       nthreads: Optional[int] = None):
+    """fp64 rows for E4M3 inputs: element value = decoded E4M3 * its tensor's scale.
+
+    Returns (out, lse, err): out is the exact output before output quantization
+    (apply o_scale and ``e4m3_encode`` for the FP8 result), err the standard
+    deviation scale of the error that rounding P to E4M3 may add to each output
+    element (see the C file).  Shapes as in ``attention_rows``.
+    """
+    lib = _load()
+    qb, kb, vb = _bytes(q), _bytes(k), _bytes(v)
+    cq = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int32))
+    ck = np.ascontiguousarray(np.asarray(cu_k, dtype=np.int32))
+    batch = len(cq) - 1
+    total_q = int(cq[-1])
+    if rows is None:
+        n = total_q * H
+        tok_p = head_p = None
+    else:
+        rows = np.asarray(rows)
+        tok = np.ascontiguousarray(rows[:, 0].astype(np.int64))
+        hd = np.ascontiguousarray(rows[:, 1].astype(np.int32))
+        n = len(tok)
+        tok_p, head_p = tok.ctypes.data, hd.ctypes.data
+    out = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    err = np.zeros((n, D), dtype=np.float64)
+    rc = lib.oracle_varlen_attention_rows_fp8(
+        qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, float(q_scale), float(k_scale),
+        float(v_scale), cq.ctypes.data, ck.ctypes.data, batch, H, H_kv, D, int(bool(causal)),
+        int(window), tok_p, head_p, n, out.ctypes.data, lse.ctypes.data, err.ctypes.data,
+        int(nthreads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_varlen_attention_rows_fp8 failed with code {rc}")
+    if rows is None:
+        return out.reshape(total_q, H, D), lse.reshape(total_q, H), err.reshape(total_q, H, D)
+    return out, lse, err

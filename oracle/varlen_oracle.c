@@ -40,6 +40,15 @@
  * arithmetic is double.  Rows are independent, so threads split the list of
  * requested (token, head) rows; nothing is blocked, fused or reordered
  * inside a row.
+ *
+ * FP8 inputs (boostr flash.rs, FlashAttentionOps::flash_attention_fwd_fp8:
+ * per-tensor dequantization scales q_scale, k_scale, v_scale take FP8 to
+ * FP32, o_scale takes the FP32 output to FP8, accumulation is FP32) are
+ * decoded here from the E4M3 format definition and multiplied by their
+ * scale, exactly, in double; the attention itself is the same definition.
+ * Readings: the FP8 format is E4M3 (the pages do not name one); o_scale
+ * multiplies the output on its way to FP8 (the FP32 -> FP8 direction the
+ * pages give it), with round-to-nearest-even and saturation at +-448.
  */
 #include <math.h>
 #include <pthread.h>
@@ -52,6 +61,48 @@ static double bf16_bits_to_double(uint16_t bits) {
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
+}
+
+/* E4M3 (the "FN" variant of the OCP 8-bit floating-point formats): one sign
+ * bit, four exponent bits with bias 7, three mantissa bits.  Exponent field 0
+ * holds the subnormals (m / 8) * 2^-6; exponent 15 with mantissa 7 is NaN;
+ * there are no infinities, so the largest finite magnitude is 1.75 * 2^8 = 448. */
+double oracle_e4m3_to_double(uint8_t b) {
+    const int sign = b >> 7, e = (b >> 3) & 15, m = b & 7;
+    double x;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) x = ldexp((double)m, -9);
+    else x = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -x : x;
+}
+
+/* Nearest E4M3 value of x, ties to the even mantissa; magnitudes of 448 and
+ * more give 448 (saturation), NaN gives NaN.  Written as a search over the
+ * non-negative finite codes 0x00..0x7E, whose values increase with the code. */
+uint8_t oracle_double_to_e4m3(double x) {
+    if (isnan(x)) return 0x7F;
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    const double a = fabs(x);
+    if (a >= 448.0) return sign | 0x7E;
+    int lo = 0;
+    for (int c = 1; c <= 0x7E; ++c)
+        if (oracle_e4m3_to_double((uint8_t)c) <= a) lo = c;
+    const double vl = oracle_e4m3_to_double((uint8_t)lo);
+    const double vh = oracle_e4m3_to_double((uint8_t)(lo + 1));
+    int pick;
+    if (a - vl < vh - a) pick = lo;
+    else if (a - vl > vh - a) pick = lo + 1;
+    else pick = (lo & 1) ? lo + 1 : lo;
+    return (uint8_t)(sign | pick);
+}
+
+/* element e of a packed tensor, widened to double and multiplied by its scale */
+typedef double (*decode_fn)(const void* base, size_t e);
+static double decode_bf16(const void* base, size_t e) {
+    return bf16_bits_to_double(((const uint16_t*)base)[e]);
+}
+static double decode_e4m3(const void* base, size_t e) {
+    return oracle_e4m3_to_double(((const uint8_t*)base)[e]);
 }
 
 /* Sequence b owning packed query token t: the b with cu_q[b] <= t < cu_q[b+1]. */
@@ -78,7 +129,10 @@ static int key_visible(int64_t i, int64_t j, int64_t L_q, int64_t L_k,
 }
 
 typedef struct {
-    const uint16_t *q, *k, *v;
+    const void *q, *k, *v;
+    decode_fn decode;
+    double q_scale, k_scale, v_scale;
+    double* err; /* optional [n_rows, D]: P-rounding error scale, see below */
     const int32_t *cu_q, *cu_k;
     const int32_t* seqused_k; /* NULL => every row of the sequence's range is a key */
     int batch, H, H_kv, D, causal, window;
@@ -90,7 +144,10 @@ typedef struct {
     int64_t max_lk;
 } job_t;
 
-static void one_row(const job_t* jb, int64_t r, double* s) {
+/* One output row.  `decode` is passed as a constant by each caller below, so
+ * the compiler specialises this function per input format. */
+static inline __attribute__((always_inline)) void one_row(const job_t* jb, int64_t r, double* s,
+                                                          decode_fn decode) {
     int64_t t;
     int h;
     if (jb->row_token) { t = jb->row_token[r]; h = jb->row_head[r]; }
@@ -107,22 +164,25 @@ static void one_row(const job_t* jb, int64_t r, double* s) {
     const int group = jb->H / jb->H_kv;
     const int hk = h / group;
     const double scale = 1.0 / sqrt((double)D);
-    const uint16_t* qrow = jb->q + ((size_t)t * jb->H + h) * D;
+    const size_t qrow = ((size_t)t * jb->H + h) * D;
     double* o = jb->out + (size_t)r * D;
+    double* err = jb->err ? jb->err + (size_t)r * D : NULL;
 
     /* scores of the visible keys; s[j] = -inf marks an invisible key */
     double m = -INFINITY;
     int64_t n_vis = 0;
     for (int64_t j = 0; j < L_k; ++j) {
         if (!key_visible(i, j, L_q, L_k, jb->causal, jb->window)) { s[j] = -INFINITY; continue; }
-        const uint16_t* krow = jb->k + (((size_t)jb->cu_k[b] + j) * jb->H_kv + hk) * D;
+        const size_t krow = (((size_t)jb->cu_k[b] + j) * jb->H_kv + hk) * D;
         double dot = 0.0;
-        for (int d = 0; d < D; ++d) dot += bf16_bits_to_double(qrow[d]) * bf16_bits_to_double(krow[d]);
+        for (int d = 0; d < D; ++d)
+            dot += (decode(jb->q, qrow + d) * jb->q_scale) * (decode(jb->k, krow + d) * jb->k_scale);
         s[j] = dot * scale;
         if (s[j] > m) m = s[j];
         ++n_vis;
     }
     for (int d = 0; d < D; ++d) o[d] = 0.0;
+    if (err) for (int d = 0; d < D; ++d) err[d] = 0.0;
     if (n_vis == 0) { jb->lse[r] = -INFINITY; return; }
 
     double l = 0.0;
@@ -130,10 +190,23 @@ static void one_row(const job_t* jb, int64_t r, double* s) {
         if (s[j] == -INFINITY) continue;
         const double p = exp(s[j] - m);
         l += p;
-        const uint16_t* vrow = jb->v + (((size_t)jb->cu_k[b] + j) * jb->H_kv + hk) * D;
-        for (int d = 0; d < D; ++d) o[d] += p * bf16_bits_to_double(vrow[d]);
+        const size_t vrow = (((size_t)jb->cu_k[b] + j) * jb->H_kv + hk) * D;
+        /* When P is rounded to E4M3 before it multiplies V, p (in units of the
+         * row maximum, which is 1 here and at most 1 when the reference is an
+         * earlier, smaller maximum) moves by at most e = max(2^-4 p, 2^-10):
+         * half the spacing of E4M3 numbers relative to a normal value, or
+         * absolute among the subnormals.  Modelling each rounding error as
+         * uniform on [-e, e] and independent across keys, the output error has
+         * variance sum_j (e_j^2 / 3) v_jd^2 / l^2; err accumulates that sum. */
+        const double e = fmax(ldexp(p, -4), ldexp(1.0, -10));
+        for (int d = 0; d < D; ++d) {
+            const double vd = decode(jb->v, vrow + d) * jb->v_scale;
+            o[d] += p * vd;
+            if (err) err[d] += e * e / 3.0 * vd * vd;
+        }
     }
     for (int d = 0; d < D; ++d) o[d] /= l;
+    if (err) for (int d = 0; d < D; ++d) err[d] = sqrt(err[d]) / l;
     jb->lse[r] = m + log(l);
 }
 
@@ -141,7 +214,10 @@ static void* run_job(void* arg) {
     const job_t* jb = (const job_t*)arg;
     double* s = (double*)malloc(sizeof(double) * (size_t)(jb->max_lk > 0 ? jb->max_lk : 1));
     if (!s) return (void*)1;
-    for (int64_t r = jb->row_begin; r < jb->row_end; ++r) one_row(jb, r, s);
+    if (jb->decode == decode_e4m3)
+        for (int64_t r = jb->row_begin; r < jb->row_end; ++r) one_row(jb, r, s, decode_e4m3);
+    else
+        for (int64_t r = jb->row_begin; r < jb->row_end; ++r) one_row(jb, r, s, decode_bf16);
     free(s);
     return NULL;
 }
@@ -160,12 +236,13 @@ static void* run_job(void* arg) {
  * out:         [n_rows, D] doubles; lse: [n_rows] doubles.
  * Returns 0, or -1 on an argument error, -2 on an allocation failure.
  */
-int oracle_varlen_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                 const int32_t* cu_q, const int32_t* cu_k,
-                                 const int32_t* seqused_k, int batch,
-                                 int H, int H_kv, int D, int causal, int window,
-                                 const int64_t* row_token, const int32_t* row_head,
-                                 int64_t n_rows, double* out, double* lse, int nthreads) {
+static int attention_rows(const void* q, const void* k, const void* v, decode_fn decode,
+                          double q_scale, double k_scale, double v_scale,
+                          const int32_t* cu_q, const int32_t* cu_k,
+                          const int32_t* seqused_k, int batch,
+                          int H, int H_kv, int D, int causal, int window,
+                          const int64_t* row_token, const int32_t* row_head,
+                          int64_t n_rows, double* out, double* lse, double* err, int nthreads) {
     if (batch < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || D < 1 || window < 0) return -1;
     if (n_rows < 0 || (n_rows > 0 && (!out || !lse))) return -1;
     if (!row_token && n_rows != (int64_t)cu_q[batch] * H) return -1;
@@ -185,6 +262,9 @@ int oracle_varlen_attention_rows(const uint16_t* q, const uint16_t* k, const uin
     for (int w = 0; w < nthreads; ++w) {
         job_t* jb = &jobs[w];
         jb->q = q; jb->k = k; jb->v = v; jb->cu_q = cu_q; jb->cu_k = cu_k;
+        jb->decode = decode;
+        jb->q_scale = q_scale; jb->k_scale = k_scale; jb->v_scale = v_scale;
+        jb->err = err;
         jb->seqused_k = seqused_k;
         jb->batch = batch; jb->H = H; jb->H_kv = H_kv; jb->D = D;
         jb->causal = causal; jb->window = window;
@@ -207,4 +287,43 @@ int oracle_varlen_attention_rows(const uint16_t* q, const uint16_t* k, const uin
     free(jobs);
     free(tids);
     return rc;
+}
+
+int oracle_varlen_attention_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                 const int32_t* cu_q, const int32_t* cu_k,
+                                 const int32_t* seqused_k, int batch,
+                                 int H, int H_kv, int D, int causal, int window,
+                                 const int64_t* row_token, const int32_t* row_head,
+                                 int64_t n_rows, double* out, double* lse, int nthreads) {
+    return attention_rows(q, k, v, decode_bf16, 1.0, 1.0, 1.0, cu_q, cu_k, seqused_k, batch, H,
+                          H_kv, D, causal, window, row_token, row_head, n_rows, out, lse, NULL,
+                          nthreads);
+}
+
+/*
+ * The same rows for E4M3 inputs with per-tensor dequantization scales
+ * (element value = decoded E4M3 * scale).  out is the exact output before it
+ * is quantized (the caller applies o_scale and oracle_double_to_e4m3);
+ * err (optional, [n_rows, D]) receives the standard-deviation scale of the
+ * error that rounding P to E4M3 may add, as described in one_row.
+ */
+int oracle_varlen_attention_rows_fp8(const uint8_t* q, const uint8_t* k, const uint8_t* v,
+                                     double q_scale, double k_scale, double v_scale,
+                                     const int32_t* cu_q, const int32_t* cu_k, int batch,
+                                     int H, int H_kv, int D, int causal, int window,
+                                     const int64_t* row_token, const int32_t* row_head,
+                                     int64_t n_rows, double* out, double* lse, double* err,
+                                     int nthreads) {
+    return attention_rows(q, k, v, decode_e4m3, q_scale, k_scale, v_scale, cu_q, cu_k, NULL,
+                          batch, H, H_kv, D, causal, window, row_token, row_head, n_rows, out,
+                          lse, err, nthreads);
+}
+
+/* Element-wise E4M3 decoding / encoding of arrays (the definitions above). */
+void oracle_e4m3_decode_array(const uint8_t* in, double* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_to_double(in[i]);
+}
+
+void oracle_e4m3_encode_array(const double* in, uint8_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_double_to_e4m3(in[i]);
 }

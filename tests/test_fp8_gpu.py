@@ -1,0 +1,168 @@
+"""GPU parity of the FP8 (E4M3) forward against the fp64 oracle.
+
+The kernel rounds P to E4M3 before the tensor-core P V product, so its output
+differs from the exact attention of the dequantized inputs by more than the
+final E4M3 rounding.  The oracle returns, per output element, the standard
+deviation scale err of that P-rounding error (each p_j moves by at most
+max(2^-4 p_j, 2^-10) in units of the row maximum, modelled as independent
+uniform rounding errors).  The bar per element is
+
+  |O_gpu - O_ref| <= 6 err + 2e-3 + half an E4M3 step at |O_ref| + 6 err + 2e-3
+
+in output units (O_gpu = decoded output code / o_scale), where 2e-3 covers the
+FP32 accumulations and the exp2 approximation; logsumexp (taken from unrounded
+P) keeps the bf16 path's 1e-3.  Where every P is exactly representable (zero
+Q: all p = 1) the P term vanishes and only the output rounding remains.
+"""
+import numpy as np
+import pytest
+import torch
+
+from variable_length_flash_varlen_b200 import binding, workloads
+
+pytestmark = pytest.mark.gpu
+
+LSE_TOL = 1e-3
+SIGMAS = 6.0
+SLACK = 2e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    binding.load()
+    binding.device_status(clear=True)
+    yield
+    assert binding.device_status(clear=True) == 0, "device status word raised"
+
+
+def e4m3_half_step(a):
+    """Half the spacing of E4M3 numbers at magnitude a (subnormal spacing 2^-9)."""
+    a = np.maximum(np.abs(a), 2.0 ** -6)
+    return np.ldexp(1.0, np.floor(np.log2(a)).astype(np.int64) - 4)
+
+
+def run_fp8(wl, q8, k8, v8, sc):
+    dev = "cuda"
+    cq = torch.tensor(wl.cu_q, dtype=torch.int32, device=dev)
+    ck = torch.tensor(wl.cu_k, dtype=torch.int32, device=dev)
+    out = torch.full(q8.shape, 0x7F, dtype=torch.uint8, device=dev)   # NaN codes
+    lse = torch.full((wl.total_q, wl.H), float("nan"), dtype=torch.float32, device=dev)
+    binding.varlen_attention_fwd_fp8(q8.to(dev), k8.to(dev), v8.to(dev), cq, ck, wl.batch, wl.H,
+                                     wl.H_kv, wl.max_seqlen_q, wl.max_seqlen_k, wl.D, wl.causal,
+                                     wl.window, sc["q_scale"], sc["k_scale"], sc["v_scale"],
+                                     sc["o_scale"], out=out, lse=lse)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+def compare_fp8(oracle_lib, out8, lse, ref_o, ref_l, err, o_scale, rows=None, p_exact=False):
+    o = oracle_lib.e4m3_decode(out8.cpu().numpy()) / o_scale
+    l = lse.cpu().double().numpy()
+    if rows is not None:
+        o = o[rows[:, 0], rows[:, 1]]
+        l = l[rows[:, 0], rows[:, 1]]
+    assert not np.isnan(o).any(), "NaN (or unwritten) output code"
+    assert not np.isnan(l).any(), "NaN logsumexp"
+    neg = np.isneginf(ref_l)
+    assert np.array_equal(np.isneginf(l), neg), "-inf logsumexp rows differ"
+    p_term = 0.0 if p_exact else SIGMAS * err + SLACK
+    slack = 1e-4 if p_exact else 0.0
+    bound = p_term + slack + e4m3_half_step((np.abs(ref_o) + p_term + slack) * o_scale) / o_scale
+    excess = np.abs(o - ref_o) - bound
+    worst = float(np.max(excess)) if o.size else 0.0
+    assert worst <= 0.0, f"FP8 output beyond its bound by {worst} (max |dO| {np.max(np.abs(o - ref_o))})"
+    fin = ~neg
+    d_l = float(np.max(np.abs(l[fin] - ref_l[fin]))) if fin.any() else 0.0
+    assert d_l <= LSE_TOL, f"max |dLSE| = {d_l}"
+    return float(np.max(np.abs(o - ref_o))) if o.size else 0.0, d_l
+
+
+def oracle_fp8(oracle_lib, wl, q8, k8, v8, sc, rows=None):
+    return oracle_lib.attention_rows_fp8(q8, k8, v8, sc["q_scale"], sc["k_scale"], sc["v_scale"],
+                                         wl.cu_q, wl.cu_k, wl.H, wl.H_kv, wl.D, wl.causal,
+                                         wl.window, rows=rows)
+
+
+REDUCED = [("mha_noncausal", 0.15), ("gqa_causal", 0.05), ("sliding_window", 1 / 32),
+           ("chunked_prefill", 0.1), ("decode", 1 / 32)]
+
+
+@pytest.mark.parametrize("name,scale", REDUCED)
+def test_fp8_reduced_workloads_match_oracle(oracle_lib, name, scale):
+    wl = workloads.named(name, scale=scale)
+    q8, k8, v8, sc = workloads.make_qkv_fp8(wl)
+    out, lse = run_fp8(wl, q8, k8, v8, sc)
+    ref_o, ref_l, err = oracle_fp8(oracle_lib, wl, q8, k8, v8, sc)
+    compare_fp8(oracle_lib, out, lse, ref_o, ref_l, err, sc["o_scale"])
+
+
+FP8_EDGE = [
+    # lengths_q, lengths_k, H, H_kv, causal, window
+    ([1, 127, 128, 129, 255, 256, 257, 1], None, 4, 1, True, 0),
+    ([1, 127, 128, 129, 255, 256, 257, 1], None, 4, 1, False, 0),
+    ([100, 5, 300], [300, 5, 130], 4, 2, True, 0),       # L_q != L_k, rows with no key
+    ([0, 130, 0, 70, 3], [0, 130, 5, 70, 0], 2, 1, True, 0),
+    ([300, 200], [300, 200], 4, 4, False, 37),
+    ([200, 333], None, 16, 2, True, 0),
+    ([2000], None, 2, 1, True, 0),
+    ([256, 129], None, 4, 2, True, 0),                  # tensor ends 1 row into a tile
+    ([256, 136], None, 4, 2, False, 0),                 # ... 8 rows in
+    ([256, 191], None, 4, 2, True, 0),                  # ... 63 rows in
+    ([256, 255], None, 4, 2, False, 0),                 # ... 127 rows in
+]
+
+
+@pytest.mark.parametrize("case", FP8_EDGE)
+def test_fp8_edge_cases_match_oracle(oracle_lib, case):
+    Lq, Lk, H, Hkv, causal, W = case
+    wl = workloads.custom(Lq, Lk if Lk is not None else Lq, H, Hkv, 128, causal, W, seed=71)
+    q8, k8, v8, sc = workloads.make_qkv_fp8(wl)
+    out, lse = run_fp8(wl, q8, k8, v8, sc)
+    ref_o, ref_l, err = oracle_fp8(oracle_lib, wl, q8, k8, v8, sc)
+    compare_fp8(oracle_lib, out, lse, ref_o, ref_l, err, sc["o_scale"])
+
+
+@pytest.mark.parametrize("causal,W", [(True, 0), (False, 0), (True, 100)])
+def test_fp8_exact_p_leaves_only_output_rounding(oracle_lib, causal, W):
+    # zero Q: every visible score is 0, every P is exactly 1 in E4M3, so the
+    # output is the mean of the visible V rows up to FP32 sums and the final
+    # E4M3 rounding (this checks the V layout and the P packing order sharply)
+    L = [300, 129, 1000]
+    wl = workloads.custom(L, L, 4, 2, 128, causal, W, seed=72)
+    _, k8, v8, sc = workloads.make_qkv_fp8(wl)
+    q8 = torch.zeros((wl.total_q, wl.H, wl.D), dtype=torch.uint8)
+    out, lse = run_fp8(wl, q8, k8, v8, sc)
+    ref_o, ref_l, err = oracle_fp8(oracle_lib, wl, q8, k8, v8, sc)
+    compare_fp8(oracle_lib, out, lse, ref_o, ref_l, err, sc["o_scale"], p_exact=True)
+
+
+def test_fp8_full_size_sampled_rows(oracle_lib):
+    # the workload the benchmark times in FP8, in the same launch configuration
+    wl = workloads.named("mha_noncausal")
+    q8, k8, v8, sc = workloads.make_qkv_fp8(wl)
+    out, lse = run_fp8(wl, q8, k8, v8, sc)
+    rng = np.random.default_rng(5)
+    rows = np.stack([rng.integers(0, wl.total_q, 512), rng.integers(0, wl.H, 512)], axis=1)
+    ref_o, ref_l, err = oracle_fp8(oracle_lib, wl, q8, k8, v8, sc, rows=rows)
+    compare_fp8(oracle_lib, out, lse, ref_o, ref_l, err, sc["o_scale"], rows=rows)
+    assert not (out.cpu().numpy() == 0x7F).any(), "output rows left unwritten"
+
+
+def test_fp8_argument_errors():
+    wl = workloads.custom([10], [10], 2, 1, 64, False, 0, seed=1)
+    cq = torch.tensor(wl.cu_q, dtype=torch.int32, device="cuda")
+    q = torch.zeros((10, 2, 64), dtype=torch.uint8, device="cuda")
+    k = torch.zeros((10, 1, 64), dtype=torch.uint8, device="cuda")
+    with pytest.raises(binding.VarlenAttentionError) as e:
+        binding.varlen_attention_fwd_fp8(q, k, k, cq, cq, 1, 2, 1, 10, 10, 64, False, 0,
+                                         1.0, 1.0, 1.0, 1.0)
+    assert e.value.code == -2  # head_dim 64 is not served in E4M3
+    q = torch.zeros((10, 2, 128), dtype=torch.uint8, device="cuda")
+    k = torch.zeros((10, 1, 128), dtype=torch.uint8, device="cuda")
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        with pytest.raises(binding.VarlenAttentionError) as e:
+            binding.varlen_attention_fwd_fp8(q, k, k, cq, cq, 1, 2, 1, 10, 10, 128, False, 0,
+                                             1.0, bad, 1.0, 1.0)
+        assert e.value.code == -1

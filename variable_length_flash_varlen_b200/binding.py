@@ -27,6 +27,8 @@ SIGNATURES = {
     "varlen_attention_fwd": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_fwd_ex": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _I, _I, _P]),
     "varlen_attention_fwd_kvcache": (_I, [_P, _P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
+    "varlen_attention_fwd_fp8": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [ctypes.c_float] * 4
+                                 + [_P, _P, _P]),
     "varlen_attention_fwd_host": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_schedule": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P]),
@@ -120,6 +122,52 @@ def varlen_attention_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         rc = lib.varlen_attention_fwd_ex(*args, int(path), int(decode_split_keys),
                                          _stream_ptr(stream))
     _check(rc)
+    return out, lse
+
+
+def _fp8_bytes(name: str, t: torch.Tensor) -> torch.Tensor:
+    if t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+        raise TypeError(f"{name} must hold E4M3 values (torch.float8_e4m3fn or uint8 bit patterns)")
+    if not t.is_contiguous() or t.device.type != "cuda":
+        raise ValueError(f"{name} must be a contiguous cuda tensor")
+    return t
+
+
+def varlen_attention_fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                             cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                             batch: int, num_heads: int, num_kv_heads: int,
+                             max_seqlen_q: int, max_seqlen_k: int, head_dim: int,
+                             causal: bool, window: int, q_scale: float, k_scale: float,
+                             v_scale: float, o_scale: float,
+                             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                             stream: Optional[torch.cuda.Stream] = None
+                             ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """FP8 (E4M3) packed attention forward with per-tensor scales; returns
+    (out as E4M3 bytes [total_q, H, D] uint8, lse float32 [total_q, H])."""
+    lib = load()
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _fp8_bytes(name, t)
+    if q.dim() != 3 or q.shape[1:] != (num_heads, head_dim):
+        raise ValueError("q must be [total_q, num_heads, head_dim]")
+    if k.shape != v.shape or k.dim() != 3 or k.shape[1:] != (num_kv_heads, head_dim):
+        raise ValueError("k and v must be [total_k, num_kv_heads, head_dim]")
+    for name, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if t.dtype != torch.int32 or not t.is_contiguous() or t.device.type != "cuda":
+            raise ValueError(f"{name} must be a contiguous int32 cuda tensor")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.uint8, device=q.device)
+    _fp8_bytes("out", out)
+    if out.shape != q.shape:
+        raise ValueError("out must be shaped like q")
+    if lse is None:
+        lse = torch.empty(q.shape[0], num_heads, dtype=torch.float32, device=q.device)
+    if lse.shape != (q.shape[0], num_heads) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [total_q, num_heads] tensor")
+    _check(lib.varlen_attention_fwd_fp8(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(),
+        batch, num_heads, num_kv_heads, max_seqlen_q, max_seqlen_k, head_dim, int(bool(causal)),
+        int(window), float(q_scale), float(k_scale), float(v_scale), float(o_scale),
+        out.data_ptr(), lse.data_ptr(), _stream_ptr(stream)))
     return out, lse
 
 

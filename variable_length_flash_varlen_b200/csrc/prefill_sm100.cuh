@@ -43,6 +43,21 @@ constexpr int kStages = 2;  // K/V ring depth (tiles of kBlockN keys)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow to 2^8 before O is rescaled
 
+// Input element formats.  bf16: Q, K, V and O in bf16, P rounded to bf16 for
+// the tensor-core PV product (kind::f16, K = 16 per instruction).  E4M3:
+// Q, K, V and O in 8-bit E4M3 with per-tensor scales (boostr flash.rs,
+// FlashAttentionOps::flash_attention_fwd_fp8: FP32 accumulation inside), P
+// rounded to E4M3 (kind::f8f6f4, K = 32 per instruction).  Either way one
+// MMA step consumes 32 bytes of every operand row.
+struct ElemBf16 {
+    static constexpr int kBytes = 2;
+    static constexpr bool kFp8 = false;
+};
+struct ElemE4m3 {
+    static constexpr int kBytes = 1;
+    static constexpr bool kFp8 = true;
+};
+
 struct PrefillParams {
     const int* cu_q;
     const int* cu_k;
@@ -51,18 +66,22 @@ struct PrefillParams {
     const TileEntry* tiles;
     SchedHeader* hdr;
     int tile_capacity;  // entries the list can hold; the count read from hdr is clamped to it
-    const __nv_bfloat16* q;
-    const __nv_bfloat16* k;
-    const __nv_bfloat16* v;
-    __nv_bfloat16* out;
+    const uint8_t* q;  // element bytes of the packed tensors (bf16 or E4M3)
+    const uint8_t* k;
+    const uint8_t* v;
+    uint8_t* out;
     float* lse;
-    float scale_log2;  // log2(e) / sqrt(D)
+    float scale_log2;  // log2(e) / sqrt(D), times q_scale * k_scale for E4M3 inputs
+    float out_mul;     // 1 for bf16; v_scale * o_scale for E4M3 (dequantize V, quantize O)
 };
 
-template <int D>
+template <int D, class E>
 struct PrefillSmem {
-    static constexpr int kChunks = D / 64;          // 128-byte swizzle atoms per row
-    static constexpr int kChunkBytes = 128 * 128;   // 128 rows x 128 bytes
+    static constexpr int kRowBytes = D * E::kBytes;             // one token row of one head
+    static constexpr int kChunks = kRowBytes / 128;             // 128-byte swizzle atoms per row
+    static_assert(kChunks >= 1 && kRowBytes % 128 == 0, "rows must be whole 128-byte atoms");
+    static constexpr int kChunkCols = 128 / E::kBytes;          // elements per atom row
+    static constexpr int kChunkBytes = 128 * 128;               // 128 rows x 128 bytes
     static constexpr int kTileBytes = kChunks * kChunkBytes;
     static constexpr int kQ = 0;                    // two Q tiles
     static constexpr int kK = kQ + 2 * kTileBytes;
@@ -73,7 +92,7 @@ struct PrefillSmem {
     static constexpr int kNumBars = 3 + 4 * kStages + 12;
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag, item ring[2]
     static constexpr int kItems = kMisc + 16;          // the ring's decoded items [2]
-    // epilogue staging, per softmax warp 32 rows x 64 bytes (one 32-column block of O)
+    // epilogue staging, per softmax warp 32 rows x 64 bytes (one 64-byte column block of O)
     static constexpr int kStage = (kItems + 2 * 64 + 15) & ~15;
     static constexpr int kBytes = kStage + 8 * 2048;
     // slack for 1024-byte alignment; never below 120 KB so that at most one CTA
@@ -117,7 +136,7 @@ __device__ __forceinline__ bool takes_part(const Item& it, int x, int kt) {
 }
 
 // Tensor maps of the three inputs, each as a 2-D view [rows][heads * D] with
-// 64-column boxes and 128-byte swizzle: one with 128-row boxes for whole
+// 128-byte-wide boxes and 128-byte swizzle: one with 128-row boxes for whole
 // tiles and one with 8-row boxes (one swizzle atom high) for a tile that runs
 // past the end of the packed tensor.  The row extent of every map is only an
 // upper bound of the packed length (batch * max_seqlen; the exact total lives
@@ -134,18 +153,21 @@ struct PrefillMaps {
 // those rows of a full box); the one partial group is read with plain loads,
 // all in flight at once, and the rows after it are zero-filled.  Completion is
 // signalled on `full` (one arrival, carrying the TMA byte count).
-template <int D>
+// `src` is the tensor's first byte, `row_stride` its row pitch in bytes and
+// `col0` the head's first element column.
+template <int D, class E>
 __device__ __forceinline__ void load_tile_ragged(uint8_t* dst, const CUtensorMap* map8,
-                                                 const __nv_bfloat16* src, int row0, int T,
+                                                 const uint8_t* src, int row0, int T,
                                                  int row_stride, int col0, uint64_t* full, int lane) {
-    constexpr int kVecPerRow = D / 8;                 // 16-byte vectors per row
+    using L = PrefillSmem<D, E>;
+    constexpr int kVecPerRow = L::kRowBytes / 16;     // 16-byte vectors per row
     constexpr int kTailVec = 8 * kVecPerRow;          // one 8-row group
     constexpr int kTailPerLane = kTailVec / 32;
     const int valid = max(0, min(128, T - row0));    // rows before T (< 128 here)
     const int g8 = valid >> 3;                        // whole 8-row groups by TMA
     const int tail0 = g8 << 3;                        // first row of the partial group
     auto swz = [&](int r, int c) {
-        return dst + (c >> 3) * PrefillSmem<D>::kChunkBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+        return dst + (c >> 3) * L::kChunkBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
     };
     uint4 vals[kTailPerLane];
 #pragma unroll
@@ -155,7 +177,7 @@ __device__ __forceinline__ void load_tile_ragged(uint8_t* dst, const CUtensorMap
         vals[u] = make_uint4(0u, 0u, 0u, 0u);
         if (r < valid)
             vals[u] = *reinterpret_cast<const uint4*>(src + static_cast<size_t>(row0 + r) * row_stride +
-                                                      col0 + c * 8);
+                                                      static_cast<size_t>(col0) * E::kBytes + c * 16);
     }
 #pragma unroll
     for (int u = 0; u < kTailPerLane; ++u) {
@@ -170,11 +192,11 @@ __device__ __forceinline__ void load_tile_ragged(uint8_t* dst, const CUtensorMap
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-        mbar_arrive_expect_tx(full, static_cast<uint32_t>(g8 * PrefillSmem<D>::kChunks * 1024));
+        mbar_arrive_expect_tx(full, static_cast<uint32_t>(g8 * L::kChunks * 1024));
         for (int g = 0; g < g8; ++g) {
 #pragma unroll
-            for (int c = 0; c < PrefillSmem<D>::kChunks; ++c)
-                tma_load_2d(dst + c * PrefillSmem<D>::kChunkBytes + g * 1024, map8, col0 + c * 64,
+            for (int c = 0; c < L::kChunks; ++c)
+                tma_load_2d(dst + c * L::kChunkBytes + g * 1024, map8, col0 + c * L::kChunkCols,
                             row0 + g * 8, full);
         }
     }
@@ -182,35 +204,37 @@ __device__ __forceinline__ void load_tile_ragged(uint8_t* dst, const CUtensorMap
 }
 
 // Whole warp: one 128-row tile into `dst`, completion signalled on `full`.
-template <int D>
+template <int D, class E>
 __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, const CUtensorMap* map8,
-                                          const __nv_bfloat16* src, int row0, int T, int row_stride,
+                                          const uint8_t* src, int row0, int T, int row_stride,
                                           int col0, uint64_t* full, int lane) {
+    using L = PrefillSmem<D, E>;
     if (row0 + 128 <= T) {
         if (lane == 0) {
-            mbar_arrive_expect_tx(full, PrefillSmem<D>::kTileBytes);
+            mbar_arrive_expect_tx(full, L::kTileBytes);
 #pragma unroll
-            for (int c = 0; c < PrefillSmem<D>::kChunks; ++c)
-                tma_load_2d(dst + c * PrefillSmem<D>::kChunkBytes, map, col0 + c * 64, row0, full);
+            for (int c = 0; c < L::kChunks; ++c)
+                tma_load_2d(dst + c * L::kChunkBytes, map, col0 + c * L::kChunkCols, row0, full);
         }
         __syncwarp();
     } else {
-        load_tile_ragged<D>(dst, map8, src, row0, T, row_stride, col0, full, lane);
+        load_tile_ragged<D, E>(dst, map8, src, row0, T, row_stride, col0, full, lane);
     }
 }
 
-template <int D>
+template <int D, class E>
 __device__ __forceinline__ void store_row_zero(const PrefillParams& p, size_t out_row) {
-    uint4* o4 = reinterpret_cast<uint4*>(p.out + out_row * D);
+    // zero is all-zero bits in both formats
+    uint4* o4 = reinterpret_cast<uint4*>(p.out + out_row * (D * E::kBytes));
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) o4[c] = make_uint4(0u, 0u, 0u, 0u);
+    for (int c = 0; c < D * E::kBytes / 16; ++c) o4[c] = make_uint4(0u, 0u, 0u, 0u);
     p.lse[out_row] = -INFINITY;
 }
 
-template <int D>
+template <int D, class E>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams p) {
-    using L = PrefillSmem<D>;
+    using L = PrefillSmem<D, E>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
@@ -277,7 +301,7 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
     if (warp == kLoadWarp) {
         // ------------------------------------------------------------ producer
         const int T_q = p.cu_q[p.batch], T_k = p.cu_k[p.batch];
-        const int q_stride = p.H * D, kv_stride = p.H_kv * D;
+        const int q_stride = p.H * D * E::kBytes, kv_stride = p.H_kv * D * E::kBytes;  // bytes
         uint32_t items_done = 0, q_issued[2] = {0, 0}, k_issued = 0, v_issued = 0, ring = 0;
         bool ok = true;
         for (;;) {
@@ -306,7 +330,7 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
                 if (it.hi_h[x] > it.lo_h[x]) {
-                    load_tile<D>(smem + L::kQ + x * L::kTileBytes, &maps.q, &maps.q8, p.q, it.q_row0 + x * kBlockM,
+                    load_tile<D, E>(smem + L::kQ + x * L::kTileBytes, &maps.q, &maps.q8, p.q, it.q_row0 + x * kBlockM,
                                  T_q, q_stride, it.h * D, &q_full[x], lane);
                     ++q_issued[x];
                 }
@@ -315,11 +339,11 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                 const int s = k_issued % kStages;
                 const uint32_t ph = (k_issued / kStages) & 1;
                 if (!(ok = mbar_wait_warp(&k_empty[s], ph ^ 1, abort_flag, status))) break;
-                load_tile<D>(smem + L::kK + s * L::kTileBytes, &maps.k, &maps.k8, p.k, it.k_row0 + kt * kBlockN,
+                load_tile<D, E>(smem + L::kK + s * L::kTileBytes, &maps.k, &maps.k8, p.k, it.k_row0 + kt * kBlockN,
                              T_k, kv_stride, it.hk * D, &k_full[s], lane);
                 ++k_issued;
                 if (!(ok = mbar_wait_warp(&v_empty[s], ph ^ 1, abort_flag, status))) break;
-                load_tile<D>(smem + L::kV + s * L::kTileBytes, &maps.v, &maps.v8, p.v, it.k_row0 + kt * kBlockN,
+                load_tile<D, E>(smem + L::kV + s * L::kTileBytes, &maps.v, &maps.v8, p.v, it.k_row0 + kt * kBlockN,
                              T_k, kv_stride, it.hk * D, &v_full[s], lane);
                 ++v_issued;
             }
@@ -346,8 +370,12 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kBlockN, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+            constexpr uint32_t idesc_qk =
+                E::kFp8 ? idesc_e4m3_f32(128, kBlockN, false) : idesc_bf16_f32(128, kBlockN, false);
+            constexpr uint32_t idesc_pv =
+                E::kFp8 ? idesc_e4m3_f32(128, D, true) : idesc_bf16_f32(128, D, true);
+            // one MMA step consumes 32 bytes of every operand row: 16 bf16 or 32 E4M3
+            constexpr int kStepKeys = 32 / E::kBytes;
             // descriptors: one high word per operand kind, low words stepped by the
             // start-address field (16-byte units)
             static_assert(L::kBar < (1 << 18), "descriptor start-address field covers 256 KB");
@@ -364,10 +392,14 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                 const uint32_t qa = q_lo + ((x * L::kTileBytes) >> 4);
                 const uint32_t kb = k_lo + ((s * L::kTileBytes) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < L::kRowBytes / 32; ++kk) {
                     const uint32_t off = ((kk >> 2) * L::kChunkBytes + (kk & 3) * 32) >> 4;
-                    mma_ss_lh<idesc_qk>(tmem + L::tmem_s(x), qa + off, q_hi, kb + off, k_hi,
-                                        kk > 0 ? 1u : 0u);
+                    if constexpr (E::kFp8)
+                        mma_ss_lh_f8<idesc_qk>(tmem + L::tmem_s(x), qa + off, q_hi, kb + off, k_hi,
+                                               kk > 0 ? 1u : 0u);
+                    else
+                        mma_ss_lh<idesc_qk>(tmem + L::tmem_s(x), qa + off, q_hi, kb + off, k_hi,
+                                            kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&s_full[x]);
             };
@@ -375,14 +407,23 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
             // o_done (the epilogue waits for it); earlier ones need no barrier of
             // their own: the S-ready commit of the next QK of the same half tracks
             // every MMA issued before it, this PV included.
-            // Keys [64 part, 64 part + 64) of the tile (the part-th half of P).
+            // Keys [64 part, 64 part + 64) of the tile (the part-th half of P); each
+            // step reads 32 bytes of P per row (8 tensor-memory columns) and
+            // kStepKeys rows of V.
             auto issue_pv = [&](int x, int s, bool first, bool last, int part) {
                 const uint32_t vb = v_lo + ((s * L::kTileBytes) >> 4);
+                constexpr int kSteps = (kBlockN / 2) / kStepKeys;
 #pragma unroll
-                for (int k4 = 0; k4 < kBlockN / 32; ++k4) {
-                    const int kk = part * (kBlockN / 32) + k4;
-                    mma_ts_lh<idesc_pv>(tmem + L::tmem_o(x), tmem + L::tmem_s(x) + kk * 8,
-                                        vb + ((kk * 16 * 128) >> 4), v_hi, (!first || kk > 0) ? 1u : 0u);
+                for (int k4 = 0; k4 < kSteps; ++k4) {
+                    const int kk = part * kSteps + k4;
+                    const uint32_t vk = vb + ((kk * kStepKeys * 128) >> 4);
+                    const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
+                    if constexpr (E::kFp8)
+                        mma_ts_lh_f8<idesc_pv>(tmem + L::tmem_o(x), tmem + L::tmem_s(x) + kk * 8, vk,
+                                               v_hi, acc);
+                    else
+                        mma_ts_lh<idesc_pv>(tmem + L::tmem_o(x), tmem + L::tmem_s(x) + kk * 8, vk,
+                                            v_hi, acc);
                 }
                 if (last) mma_commit(&o_done[x]);
             };
@@ -486,7 +527,7 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
             row_key_interval(i, it.L_q, it.L_k, p.causal != 0, p.window, lo, hi);
             const size_t out_row = static_cast<size_t>(it.q_row0 + x * kBlockM + row_in_tile) * p.H + it.h;
             if (it.hi_h[x] <= it.lo_h[x]) {
-                if (row_valid) store_row_zero<D>(p, out_row);
+                if (row_valid) store_row_zero<D, E>(p, out_row);
                 continue;
             }
             // keys every row of this warp sees: tiles inside [warp_lo, warp_hi] need no mask
@@ -546,22 +587,37 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                     m_ref = m_cand;
                 }
                 const float m_sub = (m_ref == -INFINITY) ? 0.f : m_ref;
-                // P = 2^(s * scale_log2 - m_ref) as bf16 pairs into S_x, 32 columns (64
-                // keys) at a time; the first 64 keys are handed over on their own so
+                // P = 2^(s * scale_log2 - m_ref) into S_x in the input format (bf16
+                // pairs or E4M3 quadruples), 64 keys at a time; the first 64 are handed over on their own so
                 // their PV starts while the second half is computed.  S_x's previous P
                 // was consumed by the PV issued before this QK.
                 float sums[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    uint32_t pk[32];
+                    if constexpr (E::kFp8) {
+                        // four E4M3 values per column: keys 64 half + [0, 64) in 16 columns
+                        uint32_t pk[16];
 #pragma unroll
-                    for (int c = 0; c < 64; c += 2) {
-                        const float p0 = ex2_approx(fmaf(s[half * 64 + c], p.scale_log2, -m_sub));
-                        const float p1 = ex2_approx(fmaf(s[half * 64 + c + 1], p.scale_log2, -m_sub));
-                        sums[(c >> 1) & 7] += p0 + p1;
-                        pk[c / 2] = pack_bf16x2(p0, p1);
+                        for (int c = 0; c < 64; c += 4) {
+                            const float p0 = ex2_approx(fmaf(s[half * 64 + c], p.scale_log2, -m_sub));
+                            const float p1 = ex2_approx(fmaf(s[half * 64 + c + 1], p.scale_log2, -m_sub));
+                            const float p2 = ex2_approx(fmaf(s[half * 64 + c + 2], p.scale_log2, -m_sub));
+                            const float p3 = ex2_approx(fmaf(s[half * 64 + c + 3], p.scale_log2, -m_sub));
+                            sums[(c >> 2) & 7] += (p0 + p1) + (p2 + p3);
+                            pk[c / 4] = pack_e4m3x4(p0, p1, p2, p3);
+                        }
+                        tmem_st16(sbase + half * 16, pk);
+                    } else {
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int c = 0; c < 64; c += 2) {
+                            const float p0 = ex2_approx(fmaf(s[half * 64 + c], p.scale_log2, -m_sub));
+                            const float p1 = ex2_approx(fmaf(s[half * 64 + c + 1], p.scale_log2, -m_sub));
+                            sums[(c >> 1) & 7] += p0 + p1;
+                            pk[c / 2] = pack_bf16x2(p0, p1);
+                        }
+                        tmem_st32(sbase + half * 32, pk);
                     }
-                    tmem_st32(sbase + half * 32, pk);
                     if (half == 0) {
                         if (!first_tile && move) {
                             // O_x holds every earlier P V: they were issued before this
@@ -596,29 +652,43 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
             // o_done), then O / l and logsumexp
             if (!(ok = mbar_wait_warp(&o_done[x], o_waits++ & 1, abort_flag, status))) break;
             tc_fence_after();
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            // O / l, times v_scale * o_scale for E4M3 (V's dequantization and the
+            // output's quantization folded into one factor)
+            const float inv_l = l > 0.f ? p.out_mul / l : 0.f;
             {
                 // every column block in flight before a single wait
                 uint32_t r[D / 32][32];
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) tmem_ld32(obase + c * 32, r[c]);
                 tmem_wait_ld();
-                // Through a per-warp shared-memory slice, one 32-column block at a time,
-                // so that each global store instruction writes eight rows x 64
-                // contiguous bytes instead of 16 bytes of 32 different rows.  The
-                // 16-byte chunk e of slice row r sits at position e ^ ((r >> 1) & 3):
-                // both the row-per-lane writes and the 8-row reads are conflict-free.
+                // Through a per-warp shared-memory slice, one 64-byte column block (32
+                // bf16 or 64 E4M3 values) at a time, so that each global store
+                // instruction writes eight rows x 64 contiguous bytes instead of 16
+                // bytes of 32 different rows.  The 16-byte chunk e of slice row r sits
+                // at position e ^ ((r >> 1) & 3): both the row-per-lane writes and the
+                // 8-row reads are conflict-free.
                 uint8_t* stage = smem + L::kStage + warp * 2048;
                 const int row_base = x * kBlockM + quarter * 32;  // first tile row of this warp
+                constexpr int kBlocks = L::kRowBytes / 64;
+                auto o_at = [&](int col) { return __uint_as_float(r[col >> 5][col & 31]) * inv_l; };
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < kBlocks; ++c) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(r[c][8 * e + 0]) * inv_l, __uint_as_float(r[c][8 * e + 1]) * inv_l);
-                        w.y = pack_bf16x2(__uint_as_float(r[c][8 * e + 2]) * inv_l, __uint_as_float(r[c][8 * e + 3]) * inv_l);
-                        w.z = pack_bf16x2(__uint_as_float(r[c][8 * e + 4]) * inv_l, __uint_as_float(r[c][8 * e + 5]) * inv_l);
-                        w.w = pack_bf16x2(__uint_as_float(r[c][8 * e + 6]) * inv_l, __uint_as_float(r[c][8 * e + 7]) * inv_l);
+                        if constexpr (E::kFp8) {
+                            const int c0 = c * 64 + e * 16;
+                            w.x = pack_e4m3x4(o_at(c0 + 0), o_at(c0 + 1), o_at(c0 + 2), o_at(c0 + 3));
+                            w.y = pack_e4m3x4(o_at(c0 + 4), o_at(c0 + 5), o_at(c0 + 6), o_at(c0 + 7));
+                            w.z = pack_e4m3x4(o_at(c0 + 8), o_at(c0 + 9), o_at(c0 + 10), o_at(c0 + 11));
+                            w.w = pack_e4m3x4(o_at(c0 + 12), o_at(c0 + 13), o_at(c0 + 14), o_at(c0 + 15));
+                        } else {
+                            const int c0 = c * 32 + e * 8;
+                            w.x = pack_bf16x2(o_at(c0 + 0), o_at(c0 + 1));
+                            w.y = pack_bf16x2(o_at(c0 + 2), o_at(c0 + 3));
+                            w.z = pack_bf16x2(o_at(c0 + 4), o_at(c0 + 5));
+                            w.w = pack_bf16x2(o_at(c0 + 6), o_at(c0 + 7));
+                        }
                         *reinterpret_cast<uint4*>(stage + lane * 64 + ((e ^ ((lane >> 1) & 3)) << 4)) = w;
                     }
                     __syncwarp();
@@ -628,7 +698,7 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                         const uint4 v = *reinterpret_cast<const uint4*>(stage + rr * 64 + ((ch ^ ((rr >> 1) & 3)) << 4));
                         if (it.qb * kBlockQ + row_base + rr < it.L_q) {
                             const size_t orow = static_cast<size_t>(it.q_row0 + row_base + rr) * p.H + it.h;
-                            *reinterpret_cast<uint4*>(p.out + orow * D + c * 32 + ch * 8) = v;
+                            *reinterpret_cast<uint4*>(p.out + orow * L::kRowBytes + c * 64 + ch * 16) = v;
                         }
                     }
                     __syncwarp();

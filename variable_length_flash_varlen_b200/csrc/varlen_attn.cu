@@ -92,12 +92,15 @@ int device_setup(int& dev, DeviceInfo*& info) {
             return fail(VA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
         g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<64>,
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<64, va::ElemBf16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::PrefillSmem<64>::kAlloc));
-    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128>,
+                                 va::PrefillSmem<64, va::ElemBf16>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128, va::ElemBf16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::PrefillSmem<128>::kAlloc));
+                                 va::PrefillSmem<128, va::ElemBf16>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128, va::ElemE4m3>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::PrefillSmem<128, va::ElemE4m3>::kAlloc));
     VA_CUDA(cudaFuncSetAttribute(va::build_schedule_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  va::kSortCapacity * 8));
@@ -134,13 +137,17 @@ cudaError_t ws_alloc(void** p, size_t bytes, cudaStream_t stream) {
     return cudaMallocFromPoolAsync(p, bytes, g_dev[dev].pool, stream);
 }
 
-// 2-D bf16 view [rows][cols] (cols contiguous), box 64 x box_rows, 128-byte swizzle.
-int make_tile_map(CUtensorMap* map, const void* base, long long cols, long long rows, int box_rows) {
+// 2-D view [rows][cols] (cols contiguous) of bf16 (elem_bytes 2) or 8-bit
+// (elem_bytes 1) elements; boxes of 128 bytes x box_rows, 128-byte swizzle.
+int make_tile_map(CUtensorMap* map, const void* base, long long cols, long long rows, int box_rows,
+                  int elem_bytes = 2) {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * elem_bytes};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+    const CUtensorMapDataType dtype =
+        elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = g_encode(map, dtype, 2, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -157,6 +164,9 @@ struct Args {
     void* out;
     float* lse;
     const int32_t* seqused_k = nullptr;  // key counts of a capacity-strided cache, or NULL
+    // E4M3 inputs and output with per-tensor scales (varlen_attention_fwd_fp8)
+    int fp8 = 0;
+    float q_scale = 1.f, k_scale = 1.f, v_scale = 1.f, o_scale = 1.f;
 };
 
 int validate(const Args& a) {
@@ -169,6 +179,15 @@ int validate(const Args& a) {
     if (a.D != 64 && a.D != 128)
         return fail(VA_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", a.D);
     if (a.window < 0) return fail(VA_ERR_INVALID_ARG, "window must be >= 0 (got %d)", a.window);
+    if (a.fp8) {
+        if (a.D != 128)
+            return fail(VA_ERR_UNSUPPORTED, "E4M3 inputs need head_dim 128 (got %d)", a.D);
+        const float sc[4] = {a.q_scale, a.k_scale, a.v_scale, a.o_scale};
+        const char* nm[4] = {"q_scale", "k_scale", "v_scale", "o_scale"};
+        for (int i = 0; i < 4; ++i)
+            if (!(std::isfinite(sc[i]) && sc[i] > 0.f))
+                return fail(VA_ERR_INVALID_ARG, "%s must be finite and > 0 (got %g)", nm[i], sc[i]);
+    }
     if (a.max_q < 0 || a.max_k < 0)
         return fail(VA_ERR_INVALID_ARG, "max_seqlen_q/k must be >= 0 (got %d, %d)", a.max_q, a.max_k);
     if (a.batch == 0 || a.max_q == 0) return VA_OK;
@@ -193,15 +212,54 @@ int make_prefill_maps(const Args& a, va::PrefillMaps* m) {
     const long long rows_k = std::max(1ll, static_cast<long long>(a.batch) * a.max_k);
     const long long cols_q = static_cast<long long>(a.H) * a.D;
     const long long cols_k = static_cast<long long>(a.H_kv) * a.D;
+    const int eb = a.fp8 ? 1 : 2;
     int rc;
-    if ((rc = make_tile_map(&m->q, a.q, cols_q, rows_q, va::kBlockM)) != VA_OK ||
-        (rc = make_tile_map(&m->k, a.k, cols_k, rows_k, va::kBlockN)) != VA_OK ||
-        (rc = make_tile_map(&m->v, a.v, cols_k, rows_k, va::kBlockN)) != VA_OK ||
-        (rc = make_tile_map(&m->q8, a.q, cols_q, rows_q, 8)) != VA_OK ||
-        (rc = make_tile_map(&m->k8, a.k, cols_k, rows_k, 8)) != VA_OK ||
-        (rc = make_tile_map(&m->v8, a.v, cols_k, rows_k, 8)) != VA_OK)
+    if ((rc = make_tile_map(&m->q, a.q, cols_q, rows_q, va::kBlockM, eb)) != VA_OK ||
+        (rc = make_tile_map(&m->k, a.k, cols_k, rows_k, va::kBlockN, eb)) != VA_OK ||
+        (rc = make_tile_map(&m->v, a.v, cols_k, rows_k, va::kBlockN, eb)) != VA_OK ||
+        (rc = make_tile_map(&m->q8, a.q, cols_q, rows_q, 8, eb)) != VA_OK ||
+        (rc = make_tile_map(&m->k8, a.k, cols_k, rows_k, 8, eb)) != VA_OK ||
+        (rc = make_tile_map(&m->v8, a.v, cols_k, rows_k, 8, eb)) != VA_OK)
         return rc;
     return VA_OK;
+}
+
+// Kernel parameters shared by both prefill entry paths (list and workspace
+// filled in by the caller).
+va::PrefillParams prefill_params(const Args& a) {
+    va::PrefillParams p;
+    p.cu_q = a.cu_q;
+    p.cu_k = a.cu_k;
+    p.seqused_k = a.seqused_k;
+    p.batch = a.batch;
+    p.H = a.H;
+    p.H_kv = a.H_kv;
+    p.causal = a.causal;
+    p.window = a.window;
+    p.q = static_cast<const uint8_t*>(a.q);
+    p.k = static_cast<const uint8_t*>(a.k);
+    p.v = static_cast<const uint8_t*>(a.v);
+    p.out = static_cast<uint8_t*>(a.out);
+    p.lse = a.lse;
+    // scores in base 2: log2(e) / sqrt(D), with the scales of Q and K folded in
+    const double qk = a.fp8 ? static_cast<double>(a.q_scale) * a.k_scale : 1.0;
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)) * qk);
+    p.out_mul = a.fp8 ? static_cast<float>(static_cast<double>(a.v_scale) * a.o_scale) : 1.f;
+    return p;
+}
+
+cudaError_t launch_prefill(const Args& a, const va::PrefillMaps& maps, const va::PrefillParams& p,
+                           int grid, cudaStream_t stream) {
+    if (a.fp8)
+        va::prefill_fwd_kernel<128, va::ElemE4m3>
+            <<<grid, va::kPrefillThreads, va::PrefillSmem<128, va::ElemE4m3>::kAlloc, stream>>>(maps, p);
+    else if (a.D == 64)
+        va::prefill_fwd_kernel<64, va::ElemBf16>
+            <<<grid, va::kPrefillThreads, va::PrefillSmem<64, va::ElemBf16>::kAlloc, stream>>>(maps, p);
+    else
+        va::prefill_fwd_kernel<128, va::ElemBf16>
+            <<<grid, va::kPrefillThreads, va::PrefillSmem<128, va::ElemBf16>::kAlloc, stream>>>(maps, p);
+    return cudaGetLastError();
 }
 
 int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
@@ -235,31 +293,13 @@ int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
         return cuda_fail(be, "schedule build launch");
     }
 
-    va::PrefillParams p;
-    p.cu_q = a.cu_q;
-    p.cu_k = a.cu_k;
-    p.seqused_k = a.seqused_k;
-    p.batch = a.batch;
-    p.H = a.H;
-    p.H_kv = a.H_kv;
-    p.causal = a.causal;
-    p.window = a.window;
+    va::PrefillParams p = prefill_params(a);
     p.tiles = tiles;
     p.hdr = hdr;
     p.tile_capacity = cap;
-    p.q = static_cast<const __nv_bfloat16*>(a.q);
-    p.k = static_cast<const __nv_bfloat16*>(a.k);
-    p.v = static_cast<const __nv_bfloat16*>(a.v);
-    p.out = static_cast<__nv_bfloat16*>(a.out);
-    p.lse = a.lse;
-    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)));
     const long long items = cap_ll * a.H;
     const int grid = static_cast<int>(std::min<long long>(dev.num_sms, items));
-    if (a.D == 64)
-        va::prefill_fwd_kernel<64><<<grid, va::kPrefillThreads, va::PrefillSmem<64>::kAlloc, stream>>>(maps, p);
-    else
-        va::prefill_fwd_kernel<128><<<grid, va::kPrefillThreads, va::PrefillSmem<128>::kAlloc, stream>>>(maps, p);
-    cudaError_t le = cudaGetLastError();
+    cudaError_t le = launch_prefill(a, maps, p, grid, stream);
     cudaFreeAsync(ws, stream);
     if (le != cudaSuccess) return cuda_fail(le, "prefill launch");
     return VA_OK;
@@ -345,6 +385,12 @@ int forward(const Args& a, int path, int split_keys, cudaStream_t stream) {
     if (path != VA_PATH_AUTO && path != VA_PATH_PREFILL && path != VA_PATH_DECODE)
         return fail(VA_ERR_INVALID_ARG, "unknown path %d", path);
     if (a.batch == 0 || a.max_q == 0) return VA_OK;
+    if (a.fp8) {
+        // E4M3 runs on the tile kernel for every query length
+        if (path == VA_PATH_DECODE)
+            return fail(VA_ERR_UNSUPPORTED, "the decode path takes bf16 inputs only");
+        path = VA_PATH_PREFILL;
+    }
     if (path == VA_PATH_AUTO) path = a.max_q == 1 ? VA_PATH_DECODE : VA_PATH_PREFILL;
     if (path == VA_PATH_DECODE && a.max_q > 1)
         return fail(VA_ERR_INVALID_ARG, "the decode path needs max_seqlen_q <= 1 (got %d)", a.max_q);
@@ -407,12 +453,15 @@ int noalloc_setup(NoAllocState*& st) {
             return fail(VA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
         g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<64>,
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<64, va::ElemBf16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::PrefillSmem<64>::kAlloc));
-    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128>,
+                                 va::PrefillSmem<64, va::ElemBf16>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128, va::ElemBf16>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::PrefillSmem<128>::kAlloc));
+                                 va::PrefillSmem<128, va::ElemBf16>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128, va::ElemE4m3>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::PrefillSmem<128, va::ElemE4m3>::kAlloc));
     VA_CUDA(cudaFuncSetAttribute(va::build_schedule_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  va::kSortCapacity * 8));
@@ -455,30 +504,12 @@ int run_prefill_noalloc(const Args& a, cudaStream_t stream) {
     cudaError_t be = cudaGetLastError();
     if (be != cudaSuccess) return cuda_fail(be, "schedule build launch");
 
-    va::PrefillParams p;
-    p.cu_q = a.cu_q;
-    p.cu_k = a.cu_k;
-    p.seqused_k = a.seqused_k;
-    p.batch = a.batch;
-    p.H = a.H;
-    p.H_kv = a.H_kv;
-    p.causal = a.causal;
-    p.window = a.window;
+    va::PrefillParams p = prefill_params(a);
     p.tiles = tiles;
     p.hdr = hdr;
     p.tile_capacity = cap;
-    p.q = static_cast<const __nv_bfloat16*>(a.q);
-    p.k = static_cast<const __nv_bfloat16*>(a.k);
-    p.v = static_cast<const __nv_bfloat16*>(a.v);
-    p.out = static_cast<__nv_bfloat16*>(a.out);
-    p.lse = a.lse;
-    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)));
     const int grid = static_cast<int>(std::min<long long>(st->num_sms, blocks * a.H));
-    if (a.D == 64)
-        va::prefill_fwd_kernel<64><<<grid, va::kPrefillThreads, va::PrefillSmem<64>::kAlloc, stream>>>(maps, p);
-    else
-        va::prefill_fwd_kernel<128><<<grid, va::kPrefillThreads, va::PrefillSmem<128>::kAlloc, stream>>>(maps, p);
-    cudaError_t le = cudaGetLastError();
+    cudaError_t le = launch_prefill(a, maps, p, grid, stream);
     if (le != cudaSuccess) return cuda_fail(le, "prefill launch");
     return VA_OK;
 }
@@ -494,6 +525,22 @@ int varlen_attention_fwd(const void* q, const void* k, const void* v, const int3
     g_last_error[0] = 0;
     Args a{q, k, v, cu_seqlens_q, cu_seqlens_k, batch, num_heads, num_kv_heads, max_seqlen_q,
            max_seqlen_k, head_dim, causal ? 1 : 0, window, out, lse};
+    return forward(a, VA_PATH_AUTO, 0, static_cast<cudaStream_t>(stream));
+}
+
+int varlen_attention_fwd_fp8(const void* q, const void* k, const void* v,
+                             const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                             int num_heads, int num_kv_heads, int max_seqlen_q, int max_seqlen_k,
+                             int head_dim, int causal, int window, float q_scale, float k_scale,
+                             float v_scale, float o_scale, void* out, float* lse, void* stream) {
+    g_last_error[0] = 0;
+    Args a{q, k, v, cu_seqlens_q, cu_seqlens_k, batch, num_heads, num_kv_heads, max_seqlen_q,
+           max_seqlen_k, head_dim, causal ? 1 : 0, window, out, lse};
+    a.fp8 = 1;
+    a.q_scale = q_scale;
+    a.k_scale = k_scale;
+    a.v_scale = v_scale;
+    a.o_scale = o_scale;
     return forward(a, VA_PATH_AUTO, 0, static_cast<cudaStream_t>(stream));
 }
 

@@ -27,6 +27,12 @@ Named workloads (all bf16, Q/K/V ~ N(0, 1), softmax scale 1/sqrt(D)):
                    diagonal at the end of the keys, H=32, H_kv=8, D=128
 Lengths come from random.Random(seed); Q, K, V (in that order) from a torch
 CPU generator seeded with the same seed, drawn in fixed-size chunks.
+
+FP8 inputs (``make_qkv_fp8``): the same N(0, 1) draws divided by a per-tensor
+scale of 2^-6 and rounded to E4M3 (torch's float8_e4m3fn conversion), so the
+codes span about +-350 of E4M3's +-448 and each element's value is code *
+2^-6; the output scale is 2^5, which keeps |O| * o_scale <= 448 for any
+output (|O| <= max |v| < 14 here).
 """
 from __future__ import annotations
 
@@ -116,6 +122,35 @@ def _randn_bf16(shape, gen: torch.Generator) -> torch.Tensor:
         stop = min(n, start + CHUNK)
         flat[start:stop] = torch.randn(stop - start, generator=gen, dtype=torch.float32).to(torch.bfloat16)
     return flat.view(*shape)
+
+
+FP8_INPUT_SCALE = 2.0 ** -6   # q_scale = k_scale = v_scale: dequantized value = code * scale
+FP8_OUTPUT_SCALE = 2.0 ** 5   # o_scale: output code = E4M3(O * o_scale)
+
+
+def _randn_e4m3(shape, gen: torch.Generator, scale: float) -> torch.Tensor:
+    """N(0, 1) / scale rounded to E4M3, as uint8 bit patterns."""
+    n = 1
+    for s in shape:
+        n *= s
+    flat = torch.empty(n, dtype=torch.uint8)
+    for start in range(0, n, CHUNK):
+        stop = min(n, start + CHUNK)
+        x = torch.randn(stop - start, generator=gen, dtype=torch.float32) / scale
+        flat[start:stop] = x.clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    return flat.view(*shape)
+
+
+def make_qkv_fp8(wl: Workload):
+    """E4M3 q [total_q, H, D], k and v [total_k, H_kv, D] (uint8 bit patterns) and the
+    four scales of the FP8 forward, drawn from wl.seed."""
+    gen = torch.Generator(device="cpu").manual_seed(wl.seed)
+    q = _randn_e4m3((wl.total_q, wl.H, wl.D), gen, FP8_INPUT_SCALE)
+    k = _randn_e4m3((wl.total_k, wl.H_kv, wl.D), gen, FP8_INPUT_SCALE)
+    v = _randn_e4m3((wl.total_k, wl.H_kv, wl.D), gen, FP8_INPUT_SCALE)
+    scales = {"q_scale": FP8_INPUT_SCALE, "k_scale": FP8_INPUT_SCALE,
+              "v_scale": FP8_INPUT_SCALE, "o_scale": FP8_OUTPUT_SCALE}
+    return q, k, v, scales
 
 
 def make_qkv(wl: Workload, device: str = "cpu"):
