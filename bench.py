@@ -289,11 +289,27 @@ def time_device_steps(fn, steps, warmup, flush_buf, world, stream):
 
 
 def run_profile_target(args, local):
-    """Run only the prefill or only the decode call (warm-up + steps) for an ncu capture."""
+    """Run only the prefill, the FP8 prefill or the decode call (warm-up + steps) for an ncu capture."""
     dev = torch.device("cuda", local)
     binding.load()
-    name = args.workload if args.only == "prefill" else "decode"
+    name = "decode" if args.only == "decode" else args.workload
     wl = workloads.named(name, scale=args.scale)
+    if args.only == "fp8":
+        q8, k8, v8, sc = workloads.make_qkv_fp8(wl)
+        d8 = [t.to(dev) for t in (q8, k8, v8)]
+        cq = torch.tensor(wl.cu_q, dtype=torch.int32, device=dev)
+        ck = torch.tensor(wl.cu_k, dtype=torch.int32, device=dev)
+        out8 = torch.empty_like(d8[0])
+        lse8 = torch.empty(wl.total_q, wl.H, dtype=torch.float32, device=dev)
+        for _ in range(args.warmup + args.steps):
+            binding.varlen_attention_fwd_fp8(*d8, cq, ck, wl.batch, wl.H, wl.H_kv, wl.max_seqlen_q,
+                                             wl.max_seqlen_k, wl.D, wl.causal, wl.window,
+                                             sc["q_scale"], sc["k_scale"], sc["v_scale"],
+                                             sc["o_scale"], out=out8, lse=lse8)
+        torch.cuda.synchronize()
+        if binding.device_status() != 0:
+            raise SystemExit("device status word raised")
+        return
     q, k, v = workloads.make_qkv(wl)
     dq, dk, dv = q.to(dev), k.to(dev), v.to(dev)
     cq = torch.tensor(wl.cu_q, dtype=torch.int32, device=dev)
@@ -489,7 +505,7 @@ def main():
     ap.add_argument("--no-clock-sampler", action="store_true")
     ap.add_argument("--scale", type=float, default=1.0,
                     help="shrink every sequence length (profiling captures of a small case)")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "fp8", "decode"], default="all",
                     help="profiling: run only one half of the step (no JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -105,15 +105,18 @@ int varlen_attention_fwd_kvcache(const void* q, const void* k, const void* v,
 /*
  * FP8 variant: the forward pass of FlashAttentionOps::flash_attention_fwd_fp8
  * (boostr flash.rs: per-tensor dequantization scales q_scale, k_scale,
- * v_scale take the FP8 inputs to FP32, o_scale takes the FP32 output to FP8,
- * FP32 accumulation inside) on the packed layout of varlen_attention_fwd.
+ * v_scale take the FP8 inputs to FP32, o_scale is the scale of the FP8
+ * output, FP32 accumulation inside) on the packed layout of
+ * varlen_attention_fwd.
  * q, k, v and out hold 8-bit E4M3 values (OCP "E4M3FN": bias 7, no
  * infinities, largest finite 448), one byte per element in the layouts of
- * the file comment; the element value is code * scale.  Scores are
- * (q_scale q).(k_scale k) / sqrt(head_dim); out = E4M3(O * o_scale) with
- * round-to-nearest-even and saturation at +-448, O the attention output of
- * the dequantized inputs (o_scale multiplies: the FP32 -> FP8 direction the
- * trait gives it); lse (f32) is the natural-log logsumexp of those scores.
+ * the file comment; every tensor's value is code * its scale, the output's
+ * included: out = E4M3(O / o_scale) with round-to-nearest-even and
+ * saturation at +-448, O the attention output of the dequantized inputs (the
+ * forward trait quantizes the output with o_scale, and the FP8 backward of
+ * the same trait dequantizes that output with the same o_scale).  Scores are
+ * (q_scale q).(k_scale k) / sqrt(head_dim); lse (f32) is the natural-log
+ * logsumexp of those scores.
  * P is rounded to E4M3 before the tensor-core P V product (its row sum is
  * taken unrounded).  head_dim must be 128 (VA_ERR_UNSUPPORTED otherwise);
  * the four scales must be finite and > 0 (VA_ERR_INVALID_ARG).  Every query

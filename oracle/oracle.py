@@ -165,7 +165,7 @@ def attention_rows_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float,
     """fp64 rows for E4M3 inputs: element value = decoded E4M3 * its tensor's scale.
 
     Returns (out, lse, err): out is the exact output before output quantization
-    (apply o_scale and ``e4m3_encode`` for the FP8 result), err the standard
+    (divide by o_scale and apply ``e4m3_encode`` for the FP8 result), err the standard
     deviation scale of the error that rounding P to E4M3 may add to each output
     element (see the C file).  Shapes as in ``attention_rows``.
     """

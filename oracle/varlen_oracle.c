@@ -43,12 +43,14 @@
  *
  * FP8 inputs (boostr flash.rs, FlashAttentionOps::flash_attention_fwd_fp8:
  * per-tensor dequantization scales q_scale, k_scale, v_scale take FP8 to
- * FP32, o_scale takes the FP32 output to FP8, accumulation is FP32) are
+ * FP32, o_scale is the scale the FP32 output is quantized with, accumulation
+ * is FP32) are
  * decoded here from the E4M3 format definition and multiplied by their
  * scale, exactly, in double; the attention itself is the same definition.
- * Readings: the FP8 format is E4M3 (the pages do not name one); o_scale
- * multiplies the output on its way to FP8 (the FP32 -> FP8 direction the
- * pages give it), with round-to-nearest-even and saturation at +-448.
+ * Readings: the FP8 format is E4M3 (the pages do not name one); the output
+ * code is O / o_scale (o_scale is the output's dequantization scale, as the
+ * FP8 backward of the same trait uses it), with round-to-nearest-even and
+ * saturation at +-448.
  */
 #include <math.h>
 #include <pthread.h>
@@ -303,7 +305,7 @@ int oracle_varlen_attention_rows(const uint16_t* q, const uint16_t* k, const uin
 /*
  * The same rows for E4M3 inputs with per-tensor dequantization scales
  * (element value = decoded E4M3 * scale).  out is the exact output before it
- * is quantized (the caller applies o_scale and oracle_double_to_e4m3);
+ * is quantized (the caller divides by o_scale and applies oracle_double_to_e4m3);
  * err (optional, [n_rows, D]) receives the standard-deviation scale of the
  * error that rounding P to E4M3 may add, as described in one_row.
  */

@@ -9,7 +9,7 @@ uniform rounding errors).  The bar per element is
 
   |O_gpu - O_ref| <= 6 err + 2e-3 + half an E4M3 step at |O_ref| + 6 err + 2e-3
 
-in output units (O_gpu = decoded output code / o_scale), where 2e-3 covers the
+in output units (O_gpu = decoded output code * o_scale), where 2e-3 covers the
 FP32 accumulations and the exp2 approximation; logsumexp (taken from unrounded
 P) keeps the bf16 path's 1e-3.  Where every P is exactly representable (zero
 Q: all p = 1) the P term vanishes and only the output rounding remains.
@@ -58,7 +58,7 @@ def run_fp8(wl, q8, k8, v8, sc):
 
 
 def compare_fp8(oracle_lib, out8, lse, ref_o, ref_l, err, o_scale, rows=None, p_exact=False):
-    o = oracle_lib.e4m3_decode(out8.cpu().numpy()) / o_scale
+    o = oracle_lib.e4m3_decode(out8.cpu().numpy()) * o_scale
     l = lse.cpu().double().numpy()
     if rows is not None:
         o = o[rows[:, 0], rows[:, 1]]
@@ -69,7 +69,7 @@ def compare_fp8(oracle_lib, out8, lse, ref_o, ref_l, err, o_scale, rows=None, p_
     assert np.array_equal(np.isneginf(l), neg), "-inf logsumexp rows differ"
     p_term = 0.0 if p_exact else SIGMAS * err + SLACK
     slack = 1e-4 if p_exact else 0.0
-    bound = p_term + slack + e4m3_half_step((np.abs(ref_o) + p_term + slack) * o_scale) / o_scale
+    bound = p_term + slack + e4m3_half_step((np.abs(ref_o) + p_term + slack) / o_scale) * o_scale
     excess = np.abs(o - ref_o) - bound
     worst = float(np.max(excess)) if o.size else 0.0
     assert worst <= 0.0, f"FP8 output beyond its bound by {worst} (max |dO| {np.max(np.abs(o - ref_o))})"

@@ -1,7 +1,7 @@
 """Pins for the FP8 part of the fp64 oracle (CPU only).
 
 The FP8 forward (boostr flash.rs, FlashAttentionOps::flash_attention_fwd_fp8:
-dequantization scales q/k/v_scale, output quantization scale o_scale, FP32
+dequantization scales q/k/v_scale, output scale o_scale, FP32
 accumulation) adds three things to the oracle, each checked here against
 something other than itself:
   * the E4M3 codec: every one of the 256 codes against torch's

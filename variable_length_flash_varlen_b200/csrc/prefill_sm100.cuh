@@ -17,7 +17,14 @@
 //               shared memory (8-row boxes and one group of plain loads for
 //               a tile that runs past the end of the packed tensor)
 // Tensor memory (512 columns): S_0 at 0, S_1 at 128 (P_h aliases the first
-// 64 columns of S_h), O_0 at 256, O_1 at 256 + D.
+// 64 columns of S_h, or 32 for E4M3), O_0 at 256, O_1 at 256 + D.
+//
+// Two element formats share this code (the ElemBf16 / ElemE4m3 traits):
+// bf16 inputs and output (kind::f16 MMAs), and E4M3 inputs and output with
+// per-tensor scales (kind::f8f6f4 MMAs; the FP8 forward of boostr flash.rs,
+// FlashAttentionOps::flash_attention_fwd_fp8), where the Q and K scales are
+// folded into the score scale and the V and output scales into the
+// epilogue's 1 / l.
 //
 // The recurrence is the tiled one of realizar 0.8.4 attention.rs, IMP-111
 // (online_softmax / tiled_single_head_attention): running max, running sum
@@ -39,7 +46,6 @@ namespace va {
 constexpr int kPrefillThreads = 320;
 constexpr int kMmaWarp = 8;
 constexpr int kLoadWarp = 9;
-constexpr int kStages = 2;  // K/V ring depth (tiles of kBlockN keys)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow to 2^8 before O is rescaled
 
@@ -72,7 +78,7 @@ struct PrefillParams {
     uint8_t* out;
     float* lse;
     float scale_log2;  // log2(e) / sqrt(D), times q_scale * k_scale for E4M3 inputs
-    float out_mul;     // 1 for bf16; v_scale * o_scale for E4M3 (dequantize V, quantize O)
+    float out_mul;     // 1 for bf16; v_scale / o_scale for E4M3 (dequantize V, quantize O)
 };
 
 template <int D, class E>
@@ -83,6 +89,9 @@ struct PrefillSmem {
     static constexpr int kChunkCols = 128 / E::kBytes;          // elements per atom row
     static constexpr int kChunkBytes = 128 * 128;               // 128 rows x 128 bytes
     static constexpr int kTileBytes = kChunks * kChunkBytes;
+    // K/V ring depth (tiles of kBlockN keys): E4M3 tiles are half the size, so
+    // the same shared memory holds twice the stages
+    static constexpr int kStages = E::kFp8 ? 4 : 2;
     static constexpr int kQ = 0;                    // two Q tiles
     static constexpr int kK = kQ + 2 * kTileBytes;
     static constexpr int kV = kK + kStages * kTileBytes;
@@ -242,10 +251,10 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
     uint64_t* q_full = bars + 0;  // [2]
     uint64_t* q_empty = bars + 2;
     uint64_t* k_full = bars + 3;
-    uint64_t* k_empty = k_full + kStages;
-    uint64_t* v_full = k_empty + kStages;
-    uint64_t* v_empty = v_full + kStages;
-    uint64_t* s_full = v_empty + kStages;  // [2]
+    uint64_t* k_empty = k_full + L::kStages;
+    uint64_t* v_full = k_empty + L::kStages;
+    uint64_t* v_empty = v_full + L::kStages;
+    uint64_t* s_full = v_empty + L::kStages;  // [2]
     uint64_t* p_half = s_full + 2;         // [2], P of the tile's first 64 keys stored
     uint64_t* p_full = p_half + 2;         // [2], all of P stored
     uint64_t* o_done = p_full + 2;         // [2]
@@ -271,7 +280,7 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
             mbar_init(&item_empty[x], 1 + 8);  // the MMA lane and the eight softmax warps
         }
         mbar_init(q_empty, 1);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < L::kStages; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&k_empty[s], 1);
             mbar_init(&v_full[s], 1);
@@ -289,6 +298,9 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
         prefetch_tensormap(&maps.k);
         prefetch_tensormap(&maps.v);
     }
+    // the set-up above overlaps the schedule build (programmatic dependent
+    // launch); everything below reads the list it writes
+    grid_dependency_wait();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -336,8 +348,8 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                 }
             }
             for (int kt = it.lo; kt < it.hi; ++kt) {
-                const int s = k_issued % kStages;
-                const uint32_t ph = (k_issued / kStages) & 1;
+                const int s = k_issued % L::kStages;
+                const uint32_t ph = (k_issued / L::kStages) & 1;
                 if (!(ok = mbar_wait_warp(&k_empty[s], ph ^ 1, abort_flag, status))) break;
                 load_tile<D, E>(smem + L::kK + s * L::kTileBytes, &maps.k, &maps.k8, p.k, it.k_row0 + kt * kBlockN,
                              T_k, kv_stride, it.hk * D, &k_full[s], lane);
@@ -360,9 +372,9 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
             };
             drain(&q_full[0], q_issued[0]);
             drain(&q_full[1], q_issued[1]);
-            for (int s = 0; s < kStages; ++s) {
-                const uint32_t nk = k_issued > (uint32_t)s ? (k_issued - s + kStages - 1) / kStages : 0;
-                const uint32_t nv = v_issued > (uint32_t)s ? (v_issued - s + kStages - 1) / kStages : 0;
+            for (int s = 0; s < L::kStages; ++s) {
+                const uint32_t nk = k_issued > (uint32_t)s ? (k_issued - s + L::kStages - 1) / L::kStages : 0;
+                const uint32_t nv = v_issued > (uint32_t)s ? (v_issued - s + L::kStages - 1) / L::kStages : 0;
                 drain(&k_full[s], nk);
                 drain(&v_full[s], nv);
             }
@@ -445,8 +457,8 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                 if (!ok) break;
                 // prologue: S for the first key tile
                 {
-                    const int s = kv % kStages;
-                    if (!(ok = mbar_wait(&k_full[s], (kv / kStages) & 1, abort_flag, status))) break;
+                    const int s = kv % L::kStages;
+                    if (!(ok = mbar_wait(&k_full[s], (kv / L::kStages) & 1, abort_flag, status))) break;
                     tc_fence_after();
                     for (int x = 0; x < 2; ++x)
                         if (takes_part(it, x, it.lo)) issue_qk(x, s);
@@ -457,10 +469,10 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                 for (int j = 0; j < n && ok; ++j) {
                     const int kt = it.lo + j;
                     const uint32_t kv_j = kv + j, kv_n = kv + j + 1;
-                    const int s = kv_j % kStages, s_n = kv_n % kStages;
+                    const int s = kv_j % L::kStages, s_n = kv_n % L::kStages;
                     const bool has_next = j + 1 < n;
                     bool next_k_ready = false;
-                    if (!(ok = mbar_wait(&v_full[s], (kv_j / kStages) & 1, abort_flag, status))) break;
+                    if (!(ok = mbar_wait(&v_full[s], (kv_j / L::kStages) & 1, abort_flag, status))) break;
                     for (int x = 0; x < 2 && ok; ++x) {
                         if (takes_part(it, x, kt)) {
                             const uint32_t pw = p_waits[x]++ & 1;
@@ -474,7 +486,7 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                         }
                         if (has_next && takes_part(it, x, kt + 1)) {
                             if (!next_k_ready) {
-                                if (!(ok = mbar_wait(&k_full[s_n], (kv_n / kStages) & 1, abort_flag, status)))
+                                if (!(ok = mbar_wait(&k_full[s_n], (kv_n / L::kStages) & 1, abort_flag, status)))
                                     break;
                                 tc_fence_after();
                                 next_k_ready = true;
@@ -487,7 +499,7 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                         if (!next_k_ready) {
                             // every tile of the union has a taker; this wait only keeps
                             // the ring's phases in step if that ever changes
-                            if (!(ok = mbar_wait(&k_full[s_n], (kv_n / kStages) & 1, abort_flag, status)))
+                            if (!(ok = mbar_wait(&k_full[s_n], (kv_n / L::kStages) & 1, abort_flag, status)))
                                 break;
                         }
                         mma_commit(&k_empty[s_n]);
@@ -652,7 +664,7 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
             // o_done), then O / l and logsumexp
             if (!(ok = mbar_wait_warp(&o_done[x], o_waits++ & 1, abort_flag, status))) break;
             tc_fence_after();
-            // O / l, times v_scale * o_scale for E4M3 (V's dequantization and the
+            // O / l, times v_scale / o_scale for E4M3 (V's dequantization and the
             // output's quantization folded into one factor)
             const float inv_l = l > 0.f ? p.out_mul / l : 0.f;
             {

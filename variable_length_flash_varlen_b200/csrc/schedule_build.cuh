@@ -54,6 +54,9 @@ build_schedule_kernel(const int* __restrict__ cu_q, const int* __restrict__ cu_k
     extern __shared__ unsigned long long keys[];
     __shared__ int red[32];
     const int tid = threadIdx.x;
+    // the attention kernel that reads this list may start its set-up now; it
+    // waits for this grid's completion before its first read of the list
+    grid_launch_dependents();
 
     int local = 0;
     for (int b = tid; b < batch; b += blockDim.x) {

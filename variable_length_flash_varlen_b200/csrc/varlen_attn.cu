@@ -244,22 +244,36 @@ va::PrefillParams prefill_params(const Args& a) {
     // scores in base 2: log2(e) / sqrt(D), with the scales of Q and K folded in
     const double qk = a.fp8 ? static_cast<double>(a.q_scale) * a.k_scale : 1.0;
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)) * qk);
-    p.out_mul = a.fp8 ? static_cast<float>(static_cast<double>(a.v_scale) * a.o_scale) : 1.f;
+    // E4M3 output code = O / o_scale (o_scale is the output's dequantization scale)
+    p.out_mul = a.fp8 ? static_cast<float>(static_cast<double>(a.v_scale) / a.o_scale) : 1.f;
     return p;
 }
 
+// The prefill kernel follows the schedule build on the same stream as a
+// programmatic dependent launch: its CTAs may start (barriers, tensor memory,
+// tensor-map prefetch) while the build still runs, and wait for the build's
+// completion before reading the list.
 cudaError_t launch_prefill(const Args& a, const va::PrefillMaps& maps, const va::PrefillParams& p,
                            int grid, cudaStream_t stream) {
-    if (a.fp8)
-        va::prefill_fwd_kernel<128, va::ElemE4m3>
-            <<<grid, va::kPrefillThreads, va::PrefillSmem<128, va::ElemE4m3>::kAlloc, stream>>>(maps, p);
-    else if (a.D == 64)
-        va::prefill_fwd_kernel<64, va::ElemBf16>
-            <<<grid, va::kPrefillThreads, va::PrefillSmem<64, va::ElemBf16>::kAlloc, stream>>>(maps, p);
-    else
-        va::prefill_fwd_kernel<128, va::ElemBf16>
-            <<<grid, va::kPrefillThreads, va::PrefillSmem<128, va::ElemBf16>::kAlloc, stream>>>(maps, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(va::kPrefillThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (a.fp8) {
+        cfg.dynamicSmemBytes = va::PrefillSmem<128, va::ElemE4m3>::kAlloc;
+        return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<128, va::ElemE4m3>, maps, p);
+    }
+    if (a.D == 64) {
+        cfg.dynamicSmemBytes = va::PrefillSmem<64, va::ElemBf16>::kAlloc;
+        return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<64, va::ElemBf16>, maps, p);
+    }
+    cfg.dynamicSmemBytes = va::PrefillSmem<128, va::ElemBf16>::kAlloc;
+    return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<128, va::ElemBf16>, maps, p);
 }
 
 int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {

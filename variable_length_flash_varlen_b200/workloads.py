@@ -31,8 +31,8 @@ CPU generator seeded with the same seed, drawn in fixed-size chunks.
 FP8 inputs (``make_qkv_fp8``): the same N(0, 1) draws divided by a per-tensor
 scale of 2^-6 and rounded to E4M3 (torch's float8_e4m3fn conversion), so the
 codes span about +-350 of E4M3's +-448 and each element's value is code *
-2^-6; the output scale is 2^5, which keeps |O| * o_scale <= 448 for any
-output (|O| <= max |v| < 14 here).
+2^-6; the output scale is 2^-5 (output code = O / o_scale), which keeps
+|O| / o_scale <= 448 for any output (|O| <= max |v| < 14 here).
 """
 from __future__ import annotations
 
@@ -125,7 +125,7 @@ def _randn_bf16(shape, gen: torch.Generator) -> torch.Tensor:
 
 
 FP8_INPUT_SCALE = 2.0 ** -6   # q_scale = k_scale = v_scale: dequantized value = code * scale
-FP8_OUTPUT_SCALE = 2.0 ** 5   # o_scale: output code = E4M3(O * o_scale)
+FP8_OUTPUT_SCALE = 2.0 ** -5  # o_scale: output code = E4M3(O / o_scale)
 
 
 def _randn_e4m3(shape, gen: torch.Generator, scale: float) -> torch.Tensor:
