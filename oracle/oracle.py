@@ -17,6 +17,10 @@ FlashAttentionOps::flash_attention_fwd_fp8); ``e4m3_decode`` /
 ``e4m3_encode`` are the format's definition (round to nearest even,
 saturating at +-448) written out in the same C file.
 
+``attention_bwd`` is the backward pass of the same definition (dq, dk, dv of
+sum(dout * out), boostr varlen_attention.rs VarLenAttentionOps::
+varlen_attention_bwd), in fp64.
+
 ``schedule`` (in ``oracle/schedule.py``) is the CPU statement of the tile
 work list the GPU scheduler must reproduce bit-exactly.
 """
@@ -59,6 +63,9 @@ def _load():
         f8.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_double] * 3 + [ctypes.c_void_p] * 2 + [
             ctypes.c_int] * 6 + [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64] + [
             ctypes.c_void_p] * 3 + [ctypes.c_int]
+        bw = lib.oracle_varlen_attention_bwd
+        bw.restype = ctypes.c_int
+        bw.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 6 + [ctypes.c_void_p] * 3 + [ctypes.c_int]
         for name in ("oracle_e4m3_decode_array", "oracle_e4m3_encode_array"):
             getattr(lib, name).restype = None
             getattr(lib, name).argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64]
@@ -197,3 +204,26 @@ def attention_rows_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float,
     if rows is None:
         return out.reshape(total_q, H, D), lse.reshape(total_q, H), err.reshape(total_q, H, D)
     return out, lse, err
+
+
+def attention_bwd(q, k, v, dout, cu_q: Sequence[int], cu_k: Sequence[int], H: int, H_kv: int,
+                  D: int, causal: bool, window: int = 0, nthreads: Optional[int] = None):
+    """fp64 gradients (dq [total_q, H, D], dk and dv [total_k, H_kv, D]) of
+    sum(dout * out) for the forward above; inputs bf16 (torch or uint16 bits)."""
+    lib = _load()
+    qb, kb, vb, db = _bits(q), _bits(k), _bits(v), _bits(dout)
+    cq = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int32))
+    ck = np.ascontiguousarray(np.asarray(cu_k, dtype=np.int32))
+    batch = len(cq) - 1
+    tq, tk = int(cq[-1]), int(ck[-1])
+    dq = np.zeros((tq, H, D), dtype=np.float64)
+    dk = np.zeros((tk, H_kv, D), dtype=np.float64)
+    dv = np.zeros((tk, H_kv, D), dtype=np.float64)
+    rc = lib.oracle_varlen_attention_bwd(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data,
+                                         db.ctypes.data, cq.ctypes.data, ck.ctypes.data, batch,
+                                         H, H_kv, D, int(bool(causal)), int(window),
+                                         dq.ctypes.data, dk.ctypes.data, dv.ctypes.data,
+                                         int(nthreads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_varlen_attention_bwd failed with code {rc}")
+    return dq, dk, dv

@@ -329,3 +329,150 @@ void oracle_e4m3_decode_array(const uint8_t* in, double* out, int64_t n) {
 void oracle_e4m3_encode_array(const double* in, uint8_t* out, int64_t n) {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_double_to_e4m3(in[i]);
 }
+
+/*
+ * Backward pass (boostr 0.2.0 varlen_attention.rs, VarLenAttentionOps::
+ * varlen_attention_bwd: dq [total_q, H, D], dk and dv [total_k, H_kv, D]
+ * with full GQA support; boostr flash.rs, FlashAttentionOps docs, the
+ * backward consumes the logsumexp of the forward).  Gradients of
+ * L = sum_{t,h,d} dout[t,h,d] * out[t,h,d] with out the forward above,
+ * written out from the definition for each query row i of head h:
+ *   s_ij = q_i.k_j / sqrt(D) over the visible keys, P_ij = exp(s_ij - lse_i)
+ *   (lse_i recomputed here exactly), O_i = sum_j P_ij v_j,
+ *   dP_ij = dout_i.v_j, Delta_i = dout_i.O_i = sum_j P_ij dP_ij,
+ *   dS_ij = P_ij (dP_ij - Delta_i),
+ *   dq_i = sum_j dS_ij k_j / sqrt(D),
+ *   dk_j += dS_ij q_i / sqrt(D), dv_j += P_ij dout_i
+ * (dk and dv summed over the query heads of a KV head's group).  Rows with
+ * no visible key contribute nothing.  Inputs are bf16 bit patterns, all
+ * arithmetic double.  One thread per (sequence, KV head) pair; nothing is
+ * blocked or reordered inside a row.
+ */
+typedef struct {
+    const uint16_t *q, *k, *v, *dout;
+    const int32_t *cu_q, *cu_k;
+    int batch, H, H_kv, D, causal, window;
+    double *dq, *dk, *dv;
+    int64_t pair_begin, pair_end; /* (b, hk) pairs b * H_kv + hk */
+    int64_t max_lk;
+} bwd_job_t;
+
+static void* run_bwd_job(void* arg) {
+    const bwd_job_t* jb = (const bwd_job_t*)arg;
+    const int D = jb->D, G = jb->H / jb->H_kv;
+    const double scale = 1.0 / sqrt((double)D);
+    const size_t n = (size_t)(jb->max_lk > 0 ? jb->max_lk : 1);
+    double* s = (double*)malloc(sizeof(double) * n);
+    double* dp = (double*)malloc(sizeof(double) * n);
+    double* o = (double*)malloc(sizeof(double) * (size_t)D);
+    if (!s || !dp || !o) { free(s); free(dp); free(o); return (void*)1; }
+    for (int64_t pr = jb->pair_begin; pr < jb->pair_end; ++pr) {
+        const int b = (int)(pr / jb->H_kv), hk = (int)(pr % jb->H_kv);
+        const int64_t L_q = (int64_t)jb->cu_q[b + 1] - jb->cu_q[b];
+        const int64_t L_k = (int64_t)jb->cu_k[b + 1] - jb->cu_k[b];
+        for (int h = hk * G; h < (hk + 1) * G; ++h) {
+            for (int64_t i = 0; i < L_q; ++i) {
+                const size_t qrow = (((size_t)jb->cu_q[b] + i) * jb->H + h) * D;
+                double m = -INFINITY;
+                int64_t n_vis = 0;
+                for (int64_t j = 0; j < L_k; ++j) {
+                    if (!key_visible(i, j, L_q, L_k, jb->causal, jb->window)) { s[j] = -INFINITY; continue; }
+                    const size_t krow = (((size_t)jb->cu_k[b] + j) * jb->H_kv + hk) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d)
+                        dot += bf16_bits_to_double(jb->q[qrow + d]) * bf16_bits_to_double(jb->k[krow + d]);
+                    s[j] = dot * scale;
+                    if (s[j] > m) m = s[j];
+                    ++n_vis;
+                }
+                if (n_vis == 0) continue;
+                double l = 0.0;
+                for (int64_t j = 0; j < L_k; ++j)
+                    if (s[j] != -INFINITY) l += exp(s[j] - m);
+                const double lse = m + log(l);
+                /* P_ij, O_i, dP_ij, Delta_i */
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+                for (int64_t j = 0; j < L_k; ++j) {
+                    if (s[j] == -INFINITY) continue;
+                    const double p = exp(s[j] - lse);
+                    const size_t vrow = (((size_t)jb->cu_k[b] + j) * jb->H_kv + hk) * D;
+                    double dpj = 0.0;
+                    for (int d = 0; d < D; ++d) {
+                        const double vd = bf16_bits_to_double(jb->v[vrow + d]);
+                        o[d] += p * vd;
+                        dpj += bf16_bits_to_double(jb->dout[qrow + d]) * vd;
+                    }
+                    dp[j] = dpj;
+                    s[j] = p; /* s now holds P */
+                }
+                double delta = 0.0;
+                for (int d = 0; d < D; ++d) delta += bf16_bits_to_double(jb->dout[qrow + d]) * o[d];
+                /* dS and the three gradients */
+                double* dqi = jb->dq + qrow;
+                for (int64_t j = 0; j < L_k; ++j) {
+                    if (s[j] == -INFINITY) continue;
+                    const double p = s[j];
+                    const double ds = p * (dp[j] - delta);
+                    const size_t krow = (((size_t)jb->cu_k[b] + j) * jb->H_kv + hk) * D;
+                    for (int d = 0; d < D; ++d) {
+                        dqi[d] += ds * bf16_bits_to_double(jb->k[krow + d]) * scale;
+                        jb->dk[krow + d] += ds * bf16_bits_to_double(jb->q[qrow + d]) * scale;
+                        jb->dv[krow + d] += p * bf16_bits_to_double(jb->dout[qrow + d]);
+                    }
+                }
+            }
+        }
+    }
+    free(s); free(dp); free(o);
+    return NULL;
+}
+
+/*
+ * dq [total_q, H, D], dk, dv [total_k, H_kv, D] doubles, zero-initialised
+ * here.  Returns 0, -1 on an argument error, -2 on an allocation failure.
+ */
+int oracle_varlen_attention_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                const uint16_t* dout, const int32_t* cu_q, const int32_t* cu_k,
+                                int batch, int H, int H_kv, int D, int causal, int window,
+                                double* dq, double* dk, double* dv, int nthreads) {
+    if (batch < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || D < 1 || window < 0) return -1;
+    const size_t nq = (size_t)cu_q[batch] * H * D, nk = (size_t)cu_k[batch] * H_kv * D;
+    for (size_t x = 0; x < nq; ++x) dq[x] = 0.0;
+    for (size_t x = 0; x < nk; ++x) { dk[x] = 0.0; dv[x] = 0.0; }
+    int64_t max_lk = 0;
+    for (int b = 0; b < batch; ++b) {
+        int64_t lk = (int64_t)cu_k[b + 1] - cu_k[b];
+        if (lk > max_lk) max_lk = lk;
+    }
+    const int64_t pairs = (int64_t)batch * H_kv;
+    if (nthreads < 1) nthreads = 1;
+    if ((int64_t)nthreads > pairs) nthreads = (int)pairs;
+    bwd_job_t* jobs = (bwd_job_t*)calloc((size_t)nthreads, sizeof(bwd_job_t));
+    pthread_t* tids = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !tids) { free(jobs); free(tids); return -2; }
+    int rc = 0;
+    for (int w = 0; w < nthreads; ++w) {
+        bwd_job_t* jb = &jobs[w];
+        jb->q = q; jb->k = k; jb->v = v; jb->dout = dout; jb->cu_q = cu_q; jb->cu_k = cu_k;
+        jb->batch = batch; jb->H = H; jb->H_kv = H_kv; jb->D = D;
+        jb->causal = causal; jb->window = window;
+        jb->dq = dq; jb->dk = dk; jb->dv = dv;
+        jb->pair_begin = pairs * w / nthreads;
+        jb->pair_end = pairs * (w + 1) / nthreads;
+        jb->max_lk = max_lk;
+    }
+    int started = 0;
+    for (int w = 1; w < nthreads; ++w) {
+        if (pthread_create(&tids[w], NULL, run_bwd_job, &jobs[w]) != 0) { rc = -2; break; }
+        started = w;
+    }
+    if (run_bwd_job(&jobs[0]) != NULL) rc = -2;
+    for (int w = 1; w <= started; ++w) {
+        void* ret = NULL;
+        pthread_join(tids[w], &ret);
+        if (ret != NULL) rc = -2;
+    }
+    free(jobs);
+    free(tids);
+    return rc;
+}
