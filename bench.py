@@ -6,8 +6,9 @@ non-causal MHA workload (q = k lengths uniform-int in [64, 2048], H = H_kv =
 16, D = 128), with the decode-shape HBM GB/s (128 sequences of one query,
 k lengths uniform-int in [1024, 32768], H = 32, H_kv = 8, D = 128) reported
 beside it under "decode", the chunked-prefill workload under
-"chunked_prefill" and the same headline workload in FP8 (E4M3 inputs and
-output with per-tensor scales, varlen_attention_fwd_fp8) under "fp8".  A step
+"chunked_prefill", the same headline workload in FP8 (E4M3 inputs and
+output with per-tensor scales, varlen_attention_fwd_fp8) under "fp8" and its
+backward pass (varlen_attention_bwd) under "backward".  A step
 is one call of the C ABI on one batch: schedule build + prefill kernel
 (decode: split + combine kernels).
 
@@ -418,6 +419,24 @@ def run_ours(args, world, rank, local):
     fp8_peak = peak * 2.0
     del dfq, dfk, dfv, fout, flse, fq, fk, fv
 
+    # ---- backward pass on the headline workload (dq, dk, dv from the forward's out and lse)
+    gen = torch.Generator().manual_seed(workloads.WORKLOAD_SEEDS[args.workload] + 7 + rank)
+    ddo = torch.randn(wl.total_q, wl.H, wl.D, generator=gen).to(torch.bfloat16).to(dev)
+    binding.varlen_attention_fwd(dq, dk, dv, cq, ck, wl.batch, wl.H, wl.H_kv, wl.max_seqlen_q,
+                                 wl.max_seqlen_k, wl.D, wl.causal, wl.window, out=out, lse=lse)
+    gq, gk, gv = torch.empty_like(dq), torch.empty_like(dk), torch.empty_like(dv)
+
+    def bstep():
+        binding.varlen_attention_bwd(ddo, dq, dk, dv, out, lse, cq, ck, wl.batch, wl.H, wl.H_kv,
+                                     wl.max_seqlen_q, wl.max_seqlen_k, wl.D, wl.causal, wl.window,
+                                     dq=gq, dk=gk, dv=gv)
+
+    b_ms, _ = time_device_steps(bstep, args.steps, args.warmup, flush, world, stream)
+    b_max = max_over_ranks(sum(b_ms) / 1e3, world)
+    bflops = accounting.backward_flops(wl)
+    b_value = sum_over_ranks(bflops * args.steps, world) / b_max / 1e12
+    del ddo, gq, gk, gv
+
     # ---- end to end through the host-buffer entry point (pinned memory)
     qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
     cqh = torch.tensor(wl.cu_q, dtype=torch.int32)
@@ -483,6 +502,14 @@ def run_ours(args, world, rank, local):
                              "peak_kind": f"{peak_kind} bf16 burst x 2 (nominal e4m3 / bf16 ratio)",
                              "kernel": "prefill_fwd_kernel<128, E4M3> (+ schedule build, same call)"},
                 "gpu_launches": 2 * args.steps},
+        "backward": {"workload": args.workload, "entry": "varlen_attention_bwd", "value": b_value,
+                     "unit": "TFLOP/s", "ms_per_step": b_max / args.steps * 1e3,
+                     "flops_per_step_per_gpu": bflops,
+                     "roofline": {"bound": "tensor", "achieved": b_value / world, "peak": peak,
+                                  "unit": "TFLOP/s", "frac": b_value / world / peak,
+                                  "peak_kind": f"{peak_kind} bf16 burst",
+                                  "kernel": "bwd_delta + bwd_dkdv + bwd_dq (same call)"},
+                     "gpu_launches": 3 * args.steps},
         "e2e": {"value": e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,

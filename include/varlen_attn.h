@@ -132,6 +132,31 @@ int varlen_attention_fwd_fp8(const void* q, const void* k, const void* v,
                              void* stream);
 
 /*
+ * Backward pass: VarLenAttentionOps::varlen_attention_bwd of boostr 0.2.0
+ * varlen_attention.rs (argument order kept: dout, q, k, v, the forward's
+ * output and logsumexp, cu_seqlens, sizes, causal), with `window` as in the
+ * forward (FlashAttentionOps::flash_attention_bwd of flash.rs takes it) and
+ * the gradients passed in instead of returned.  Computes the gradients of
+ * sum(dout * out) for the forward of varlen_attention_fwd with the same
+ * masks:
+ *   dq [total_q, num_heads, head_dim], dk and dv [total_k, num_kv_heads,
+ *   head_dim] (GQA: summed over the query heads of each KV head), bf16.
+ * dout, q, k, v, out are bf16 in the forward's layouts, lse f32
+ * [total_q, num_heads] (natural log, -inf for rows with no visible key), all
+ * caller-owned device memory; out and lse must be the forward's results for
+ * these inputs (Delta_i = sum_d dout * out is formed from them).  Every row of
+ * dq, dk, dv inside the sequences is written (zero where no visible pair
+ * touches it).  head_dim 64 or 128; batch and num_heads <= 65535.  A delta
+ * buffer of batch * max_seqlen_q * num_heads floats is allocated and freed
+ * stream-ordered.  Asynchrony and errors as for varlen_attention_fwd.
+ */
+int varlen_attention_bwd(const void* dout, const void* q, const void* k, const void* v,
+                         const void* out, const float* lse, const int32_t* cu_seqlens_q,
+                         const int32_t* cu_seqlens_k, int batch, int num_heads, int num_kv_heads,
+                         int max_seqlen_q, int max_seqlen_k, int head_dim, int causal, int window,
+                         void* dq, void* dk, void* dv, void* stream);
+
+/*
  * Same as varlen_attention_fwd with the path forced (VA_PATH_*) and, for the
  * decode path, the number of keys per split (decode_split_keys in [32, 65536];
  * 0 = library default: the largest of 4096, 2048, ..., 256 keys that still

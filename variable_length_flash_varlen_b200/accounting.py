@@ -40,6 +40,13 @@ def attention_flops(wl: Workload) -> float:
     return 4.0 * visible_pairs(wl) * wl.D * wl.H
 
 
+def backward_flops(wl: Workload) -> float:
+    """Algorithmic FLOPs of the backward pass: 10 * visible pairs * D * H, the five
+    products S = QK^T (recomputed), dP = dO V^T, dV = P^T dO, dK = dS^T Q and
+    dQ = dS K at 2 flops per multiply-add (2.5 x the forward)."""
+    return 10.0 * visible_pairs(wl) * wl.D * wl.H
+
+
 def decode_bytes(wl: Workload) -> int:
     """Algorithmic HBM bytes of one pass: K and V once, Q, O (bf16) and LSE (f32)."""
     kv = 2 * wl.total_k * wl.H_kv * wl.D * 2

@@ -29,6 +29,7 @@ SIGNATURES = {
     "varlen_attention_fwd_kvcache": (_I, [_P, _P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_fwd_fp8": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [ctypes.c_float] * 4
                                  + [_P, _P, _P]),
+    "varlen_attention_bwd": (_I, [_P] * 8 + [_I] * 8 + [_P] * 4),
     "varlen_attention_fwd_host": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_schedule": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P]),
@@ -169,6 +170,35 @@ def varlen_attention_fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         int(window), float(q_scale), float(k_scale), float(v_scale), float(o_scale),
         out.data_ptr(), lse.data_ptr(), _stream_ptr(stream)))
     return out, lse
+
+
+def varlen_attention_bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                         out: torch.Tensor, lse: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                         cu_seqlens_k: torch.Tensor, batch: int, num_heads: int, num_kv_heads: int,
+                         max_seqlen_q: int, max_seqlen_k: int, head_dim: int, causal: bool,
+                         window: int = 0, dq: Optional[torch.Tensor] = None,
+                         dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
+                         stream: Optional[torch.cuda.Stream] = None):
+    """Backward pass on device tensors; returns (dq, dk, dv) in bf16."""
+    lib = load()
+    _check_inputs(q, k, v, cu_seqlens_q, cu_seqlens_k, num_heads, num_kv_heads, head_dim, "cuda")
+    for name, t, like in (("dout", dout, q), ("out", out, q)):
+        if t.shape != like.shape or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 tensor shaped like q")
+    if lse.shape != (q.shape[0], num_heads) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [total_q, num_heads] tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t, like in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        if t.shape != like.shape or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 tensor shaped like its input")
+    _check(lib.varlen_attention_bwd(
+        dout.data_ptr(), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+        cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), batch, num_heads, num_kv_heads,
+        max_seqlen_q, max_seqlen_k, head_dim, int(bool(causal)), int(window), dq.data_ptr(),
+        dk.data_ptr(), dv.data_ptr(), _stream_ptr(stream)))
+    return dq, dk, dv
 
 
 def varlen_attention_fwd_kvcache(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,

@@ -13,6 +13,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "backward_sm100.cuh"
 #include "decode.cuh"
 #include "prefill_sm100.cuh"
 #include "schedule_build.cuh"
@@ -104,6 +105,14 @@ int device_setup(int& dev, DeviceInfo*& info) {
     VA_CUDA(cudaFuncSetAttribute(va::build_schedule_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  va::kSortCapacity * 8));
+    VA_CUDA(cudaFuncSetAttribute(va::bwd_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::BwdSmem<64>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::bwd_dkdv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::BwdSmem<128>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::BwdSmem<64>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::bwd_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::BwdSmem<128>::kAlloc));
     VA_CUDA(cudaFuncSetAttribute(va::decode_stream_kernel<64>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  va::DecodeSmem<64>::kAlloc));
@@ -417,6 +426,92 @@ int forward(const Args& a, int path, int split_keys, cudaStream_t stream) {
 }
 
 // ---------------------------------------------------------------------------
+// Backward pass: Delta = rowsum(dout * out), then dK/dV per key tile and dQ
+// per query tile (backward_sm100.cuh).
+
+struct BwdArgs {
+    Args fwd;  // q, k, v, cu_seqlens, sizes, masks; out = the forward output, lse its logsumexp
+    const void* dout;
+    void *dq, *dk, *dv;
+};
+
+int run_backward(const BwdArgs& g, cudaStream_t stream) {
+    const Args& a = g.fwd;
+    int rc = validate(a);
+    if (rc != VA_OK) return rc;
+    const char* names[] = {"dout", "dq", "dk", "dv"};
+    const void* ptrs[] = {g.dout, g.dq, g.dk, g.dv};
+    if (a.batch > 0 && (a.max_q > 0 || a.max_k > 0)) {
+        for (int i = 0; i < 4; ++i) {
+            if (!ptrs[i]) return fail(VA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+            if (!aligned16(ptrs[i])) return fail(VA_ERR_INVALID_ARG, "%s must be 16-byte aligned", names[i]);
+        }
+    }
+    if (a.batch == 0) return VA_OK;
+    if (a.batch > 65535 || a.H > 65535)
+        return fail(VA_ERR_UNSUPPORTED, "batch and num_heads must be <= 65535 for the backward grid");
+    int dev;
+    DeviceInfo* info;
+    if ((rc = device_setup(dev, info)) != VA_OK) return rc;
+    const long long rows_q = std::max(1ll, static_cast<long long>(a.batch) * a.max_q);
+    const long long rows_k = std::max(1ll, static_cast<long long>(a.batch) * a.max_k);
+    const long long cols_q = static_cast<long long>(a.H) * a.D;
+    const long long cols_k = static_cast<long long>(a.H_kv) * a.D;
+    va::BwdMaps maps;
+    if ((rc = make_tile_map(&maps.q, a.q, cols_q, rows_q, va::kBlockM)) != VA_OK ||
+        (rc = make_tile_map(&maps.dout, g.dout, cols_q, rows_q, va::kBlockM)) != VA_OK ||
+        (rc = make_tile_map(&maps.k, a.k, cols_k, rows_k, va::kBlockN)) != VA_OK ||
+        (rc = make_tile_map(&maps.v, a.v, cols_k, rows_k, va::kBlockN)) != VA_OK ||
+        (rc = make_tile_map(&maps.q8, a.q, cols_q, rows_q, 8)) != VA_OK ||
+        (rc = make_tile_map(&maps.dout8, g.dout, cols_q, rows_q, 8)) != VA_OK ||
+        (rc = make_tile_map(&maps.k8, a.k, cols_k, rows_k, 8)) != VA_OK ||
+        (rc = make_tile_map(&maps.v8, a.v, cols_k, rows_k, 8)) != VA_OK)
+        return rc;
+    float* delta = nullptr;
+    VA_CUDA(ws_alloc(reinterpret_cast<void**>(&delta), static_cast<size_t>(rows_q) * a.H * sizeof(float),
+                     stream));
+    va::BwdParams p;
+    p.cu_q = a.cu_q;
+    p.cu_k = a.cu_k;
+    p.batch = a.batch;
+    p.H = a.H;
+    p.H_kv = a.H_kv;
+    p.causal = a.causal;
+    p.window = a.window;
+    p.q = static_cast<const uint8_t*>(a.q);
+    p.k = static_cast<const uint8_t*>(a.k);
+    p.v = static_cast<const uint8_t*>(a.v);
+    p.dout = static_cast<const uint8_t*>(g.dout);
+    p.out = static_cast<const uint8_t*>(a.out);
+    p.lse = a.lse;
+    p.delta = delta;
+    p.dq = static_cast<uint8_t*>(g.dq);
+    p.dk = static_cast<uint8_t*>(g.dk);
+    p.dv = static_cast<uint8_t*>(g.dv);
+    p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(a.D)));
+    p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)));
+    const long long delta_rows = rows_q * a.H;
+    const unsigned delta_blocks = static_cast<unsigned>((delta_rows + 7) / 8);
+    const dim3 grid_kv(static_cast<unsigned>((std::max(a.max_k, 1) + va::kBlockN - 1) / va::kBlockN),
+                       static_cast<unsigned>(a.H_kv), static_cast<unsigned>(a.batch));
+    const dim3 grid_q(static_cast<unsigned>((std::max(a.max_q, 1) + va::kBlockM - 1) / va::kBlockM),
+                      static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch));
+    if (a.D == 64) {
+        va::bwd_delta_kernel<64><<<delta_blocks, 256, 0, stream>>>(p);
+        va::bwd_dkdv_kernel<64><<<grid_kv, va::kBwdThreads, va::BwdSmem<64>::kAlloc, stream>>>(maps, p);
+        va::bwd_dq_kernel<64><<<grid_q, va::kBwdThreads, va::BwdSmem<64>::kAlloc, stream>>>(maps, p);
+    } else {
+        va::bwd_delta_kernel<128><<<delta_blocks, 256, 0, stream>>>(p);
+        va::bwd_dkdv_kernel<128><<<grid_kv, va::kBwdThreads, va::BwdSmem<128>::kAlloc, stream>>>(maps, p);
+        va::bwd_dq_kernel<128><<<grid_q, va::kBwdThreads, va::BwdSmem<128>::kAlloc, stream>>>(maps, p);
+    }
+    cudaError_t le = cudaGetLastError();
+    cudaFreeAsync(delta, stream);
+    if (le != cudaSuccess) return cuda_fail(le, "backward launch");
+    return VA_OK;
+}
+
+// ---------------------------------------------------------------------------
 // Entry point without allocation.  Some callers must not reach any device
 // allocator: code running inside a framework or serving runtime that owns all
 // device memory through its own allocator, or a latency-critical loop that may
@@ -556,6 +651,19 @@ int varlen_attention_fwd_fp8(const void* q, const void* k, const void* v,
     a.v_scale = v_scale;
     a.o_scale = o_scale;
     return forward(a, VA_PATH_AUTO, 0, static_cast<cudaStream_t>(stream));
+}
+
+int varlen_attention_bwd(const void* dout, const void* q, const void* k, const void* v,
+                         const void* out, const float* lse, const int32_t* cu_seqlens_q,
+                         const int32_t* cu_seqlens_k, int batch, int num_heads, int num_kv_heads,
+                         int max_seqlen_q, int max_seqlen_k, int head_dim, int causal, int window,
+                         void* dq, void* dk, void* dv, void* stream) {
+    g_last_error[0] = 0;
+    BwdArgs g{Args{q, k, v, cu_seqlens_q, cu_seqlens_k, batch, num_heads, num_kv_heads,
+                   max_seqlen_q, max_seqlen_k, head_dim, causal ? 1 : 0, window,
+                   const_cast<void*>(out), const_cast<float*>(lse)},
+              dout, dq, dk, dv};
+    return run_backward(g, static_cast<cudaStream_t>(stream));
 }
 
 int varlen_attention_fwd_kvcache(const void* q, const void* k, const void* v,
