@@ -9,30 +9,41 @@
 //   dS_ij = P_ij (dP_ij - Delta_i)
 //   dv_j = sum_i P_ij dout_i,  dk_j = sum_i dS_ij q_i / sqrt(D),
 //   dq_i = sum_j dS_ij k_j / sqrt(D).
-// Three kernels, no atomics, every output element written by one CTA:
-//   bwd_delta_kernel   Delta_i (one warp per token row and head)
+// Two kernels, no atomics, every output element written by one CTA, dQ first:
+//   bwd_dq_kernel      one CTA per (128-row query tile, query head, sequence):
+//                      Delta_i of its rows (stored for the other kernel), then
+//                      with Q and dout resident, for every visible key tile
+//                      S = Q K^T, dP = dout V^T, dS (bf16) into tensor memory,
+//                      dQ += dS K
 //   bwd_dkdv_kernel    one CTA per (key tile of 128 keys, KV head, sequence):
 //                      K and V stay in shared memory; for every query head of
 //                      the group and every 128-row query tile that sees the key
-//                      tile: S^T = K Q^T and dP^T = V dout^T on tensor cores,
-//                      P^T and dS^T (bf16) back into tensor memory, then
-//                      dV += P^T dout and dK += dS^T Q (TS form), accumulated
-//                      in tensor memory over the whole loop
-//   bwd_dq_kernel      one CTA per (128-row query tile, query head, sequence):
-//                      Q and dout stay; for every visible key tile S = Q K^T,
-//                      dP = dout V^T, dS (bf16) into tensor memory, dQ += dS K
-// Warp roles (192 threads): warps 0-3 the element-wise work and the epilogue
-// (one key row, or one query row, per thread), warp 4 the TMA producer, warp 5
-// the tensor-memory owner and MMA issuer (one lane).
+//                      tile: S^T = K Q^T, then P^T (bf16) into tensor memory
+//                      while dP^T = V dout^T runs, then dS^T (bf16) while
+//                      dV += P^T dout runs, then dK += dS^T Q (TS form), the
+//                      two accumulators in tensor memory over the whole loop
+// Warp roles (320 threads): warps 0-7 the element-wise work and the epilogue
+// (one key row, or one query row, per thread; warps w and w + 4 share a
+// tensor-memory lane quarter and take one half of the 128 columns each), warp
+// 8 the TMA producer, warp 9 the tensor-memory owner and MMA issuer (one lane).
 #pragma once
 
 #include "prefill_sm100.cuh"
 
 namespace va {
 
-constexpr int kBwdThreads = 192;
-constexpr int kBwdLoadWarp = 4;
-constexpr int kBwdMmaWarp = 5;
+constexpr int kBwdThreads = 320;
+constexpr int kBwdEwWarps = 8;
+constexpr int kBwdLoadWarp = 8;
+constexpr int kBwdMmaWarp = 9;
+
+// Where the bf16 values formed from 32-column chunk c of an f32 tile (S^T,
+// dP^T, S or dP, 128 columns) are stored: the two warps of a lane quarter
+// own chunks {0, 1} and {2, 3}, and each writes only over columns it has
+// already read itself (16 packed columns per chunk, at 0, 16 and 64, 80).
+__host__ __device__ constexpr uint32_t bwd_pcol(int c) { return (c >> 1) * 64 + (c & 1) * 16; }
+// The same place seen by the MMA that consumes it: 16 rows of K per step.
+__host__ __device__ constexpr uint32_t bwd_kcol(int kk) { return bwd_pcol(kk >> 1) + (kk & 1) * 8; }
 
 struct BwdParams {
     const int* cu_q;
@@ -44,7 +55,12 @@ struct BwdParams {
     const uint8_t* dout;  // [total_q, H, D]
     const uint8_t* out;   // forward output, [total_q, H, D]
     const float* lse;     // forward logsumexp (natural log), [total_q, H]
-    float* delta;         // [total_q, H] written by bwd_delta_kernel
+    // per (head, token): {lse * log2(e), Delta}, head-major [H][rows_cap], written by
+    // bwd_dq_kernel for every query row that sees a key, read by bwd_dkdv_kernel
+    // (128 consecutive rows of one head per query tile)
+    float2* rowinfo;
+    long long rows_cap;   // >= total_q
+
     uint8_t* dq;          // bf16 outputs
     uint8_t* dk;
     uint8_t* dv;
@@ -59,24 +75,6 @@ struct BwdMaps {
     CUtensorMap q8, dout8, k8, v8;
 };
 
-// Delta_i = sum_d dout[i, d] * out[i, d] in f32, one warp per (token, head) row.
-template <int D>
-__global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdParams p) {
-    const long long rows = static_cast<long long>(p.cu_q[p.batch]) * p.H;
-    const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    if (row >= rows) return;
-    const int lane = threadIdx.x & 31;
-    constexpr int kPer = D / 32;  // bf16 values per lane
-    const __nv_bfloat16* o = reinterpret_cast<const __nv_bfloat16*>(p.out) + row * D + lane * kPer;
-    const __nv_bfloat16* g = reinterpret_cast<const __nv_bfloat16*>(p.dout) + row * D + lane * kPer;
-    float acc = 0.f;
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) acc = fmaf(__bfloat162float(o[e]), __bfloat162float(g[e]), acc);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) p.delta[row] = acc;
-}
-
 template <int D>
 struct BwdSmem {
     using T = PrefillSmem<D, ElemBf16>;
@@ -89,8 +87,9 @@ struct BwdSmem {
     static constexpr int kRing1 = 4 * kTile;      // [2]
     static constexpr int kRows = 6 * kTile;       // [2][128] f32 lse * log2(e), [2][128] f32 Delta
     static constexpr int kBar = kRows + 4 * 128 * 4;
-    // fixed_full, ring_full[2], ring_empty[2], s_full, p_ready, acc_done
-    static constexpr int kNumBars = 8;
+    // fixed_full, ring_full[2], ring_empty[2], s_full, p_ready, acc_done, dp_full, ds_ready,
+    // p_read
+    static constexpr int kNumBars = 11;
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
@@ -105,6 +104,9 @@ struct BwdBars {
     uint64_t* s_full;
     uint64_t* p_ready;
     uint64_t* acc_done;
+    uint64_t* dp_full;   // dK/dV kernel: dP^T ready (S^T has its own s_full)
+    uint64_t* ds_ready;  // dK/dV kernel: dS^T stored
+    uint64_t* p_read;    // dK/dV kernel: the element-wise warps have loaded P^T (S^T may be overwritten)
     uint32_t* tmem_slot;
     volatile int* abort_flag;
 };
@@ -120,6 +122,9 @@ __device__ __forceinline__ BwdBars bwd_setup(uint8_t* smem, int warp) {
     r.s_full = bars + 5;
     r.p_ready = bars + 6;
     r.acc_done = bars + 7;
+    r.dp_full = bars + 8;
+    r.ds_ready = bars + 9;
+    r.p_read = bars + 10;
     r.tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     r.abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     if (threadIdx.x == 0) {
@@ -129,8 +134,11 @@ __device__ __forceinline__ BwdBars bwd_setup(uint8_t* smem, int warp) {
             mbar_init(&r.ring_empty[s], 1);
         }
         mbar_init(r.s_full, 1);
-        mbar_init(r.p_ready, 4);  // the four element-wise warps
+        mbar_init(r.p_ready, kBwdEwWarps);
         mbar_init(r.acc_done, 1);
+        mbar_init(r.dp_full, 1);
+        mbar_init(r.ds_ready, kBwdEwWarps);
+        mbar_init(r.p_read, kBwdEwWarps);
         *r.abort_flag = 0;
         fence_barrier_init();
     }
@@ -162,14 +170,15 @@ __device__ __forceinline__ void bwd_drain(uint64_t* bar, uint32_t issued, unsign
     }
 }
 
-// This thread's row (its TMEM lane) of a D-column f32 accumulator at tensor
-// memory address `taddr`, scaled by `mul`, as bf16 to dst + row * row_pitch
-// (nothing is stored when !valid; the loads still run, they are warp-wide).
-template <int D>
+// kCols columns of this thread's row (its TMEM lane) of an f32 accumulator
+// at tensor-memory address `taddr`, scaled by `mul`, as bf16 to
+// dst + row * row_pitch (nothing is stored when !valid; the loads still run,
+// they are warp-wide).
+template <int kCols>
 __device__ __forceinline__ void bwd_store_rows(uint32_t taddr, float mul, uint8_t* dst,
                                                long long row_pitch, int row, bool valid) {
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = 0; c < kCols / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(taddr + c * 32, r);
         tmem_wait_ld();
@@ -249,16 +258,21 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
             const int h = hk * G + n / n_qt, qt = qt0 + n % n_qt;
             if (!(ok = mbar_wait_warp(&bar.ring_empty[st], ((n >> 1) & 1) ^ 1, bar.abort_flag, status)))
                 break;
-            for (int r = lane; r < kBlockM; r += 32) {
-                const int i = qt * kBlockM + r;
-                float l2 = 0.f, dl = 0.f;  // rows past the sequence: masked, any finite value
-                if (i < L_q) {
-                    const float l = p.lse[static_cast<size_t>(cq + i) * p.H + h];
-                    l2 = l == -INFINITY ? 0.f : l * 1.4426950408889634f;
-                    dl = p.delta[static_cast<size_t>(cq + i) * p.H + h];
+            {
+                // the tile's 128 rows of {lse * log2(e), Delta}: four loads per lane in
+                // flight at once (rows past the sequence are masked: any finite value)
+                const float2* src = p.rowinfo + h * p.rows_cap + cq + qt * kBlockM;
+                float2 ri[kBlockM / 32];
+#pragma unroll
+                for (int u = 0; u < kBlockM / 32; ++u) {
+                    const int r = lane + 32 * u;
+                    ri[u] = qt * kBlockM + r < L_q ? src[r] : make_float2(0.f, 0.f);
                 }
-                lse_s[st * kBlockM + r] = l2;
-                dlt_s[st * kBlockM + r] = dl;
+#pragma unroll
+                for (int u = 0; u < kBlockM / 32; ++u) {
+                    lse_s[st * kBlockM + lane + 32 * u] = ri[u].x;
+                    dlt_s[st * kBlockM + lane + 32 * u] = ri[u].y;
+                }
             }
             __syncwarp();
             load_tile<D, ElemBf16>(smem + L::kRing0 + st * L::kTile, &maps.q, &maps.q8, p.q,
@@ -287,37 +301,61 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
             const uint32_t hi_k = static_cast<uint32_t>(dk_ >> 32), hi_mn = static_cast<uint32_t>(dq_mn >> 32);
             bool ok = mbar_wait(bar.fixed_full, 0, bar.abort_flag, status);
             tc_fence_after();
-            for (int n = 0; n < n_steps && ok; ++n) {
-                const int st = n & 1;
-                if (!(ok = mbar_wait(&bar.ring_full[st], (n >> 1) & 1, bar.abort_flag, status))) break;
-                tc_fence_after();
-                const uint32_t ring = (st * L::kTile) >> 4;
-                // S^T = K Q^T and dP^T = V dout^T (K-major operands, K = D)
+            // S^T = K Q^T for step m (Q of ring stage m & 1, K-major operands, K = D)
+            auto issue_s = [&](int m) {
+                const uint32_t ring = ((m & 1) * L::kTile) >> 4;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * T::kChunkBytes + (kk & 3) * 32) >> 4;
                     mma_ss_lh<idesc_ss>(tmem + kS, static_cast<uint32_t>(dk_) + off, hi_k,
                                         static_cast<uint32_t>(dq_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
                 }
+                mma_commit(bar.s_full);
+            };
+            // Order per step n: dP^T(n), dV(n) once P^T(n) is stored, S^T(n+1) once
+            // the element-wise warps have loaded P^T(n) (it overwrites those
+            // columns; dV(n), issued before it, reads them first), dK(n) once
+            // dS^T(n) is stored.  The S^T of the next step so runs while dS^T is
+            // formed.  dP^T(n+1) overwrites dS^T(n) and follows dK(n).
+            if (ok && n_steps > 0) {
+                ok = mbar_wait(&bar.ring_full[0], 0, bar.abort_flag, status);
+                tc_fence_after();
+                if (ok) issue_s(0);
+            }
+            for (int n = 0; n < n_steps && ok; ++n) {
+                const int st = n & 1;
+                const uint32_t ring = (st * L::kTile) >> 4;
+                // dP^T = V dout^T (K-major operands, K = D)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * T::kChunkBytes + (kk & 3) * 32) >> 4;
                     mma_ss_lh<idesc_ss>(tmem + kDP, static_cast<uint32_t>(dv_) + off, hi_k,
                                         static_cast<uint32_t>(dd_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(bar.s_full);
+                mma_commit(bar.dp_full);
+                // dV += P^T dout (A from tensor memory, B MN-major, K = 128 query rows)
                 if (!(ok = mbar_wait(bar.p_ready, n & 1, bar.abort_flag, status))) break;
                 tc_fence_after();
-                // dV += P^T dout and dK += dS^T Q (A from tensor memory, B MN-major, K = 128 rows)
 #pragma unroll
-                for (int kk = 0; kk < kBlockM / 16; ++kk) {
-                    const uint32_t boff = ring + ((kk * 16 * 128) >> 4);
-                    const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-                    mma_ts_lh<idesc_ts>(tmem + kDV, tmem + kS + kk * 8,
-                                        static_cast<uint32_t>(dd_mn) + boff, hi_mn, acc);
-                    mma_ts_lh<idesc_ts>(tmem + kDK, tmem + kDP + kk * 8,
-                                        static_cast<uint32_t>(dq_mn) + boff, hi_mn, acc);
+                for (int kk = 0; kk < kBlockM / 16; ++kk)
+                    mma_ts_lh<idesc_ts>(tmem + kDV, tmem + kS + bwd_kcol(kk),
+                                        static_cast<uint32_t>(dd_mn) + ring + ((kk * 16 * 128) >> 4), hi_mn,
+                                        (n > 0 || kk > 0) ? 1u : 0u);
+                if (n + 1 < n_steps) {
+                    if (!(ok = mbar_wait(&bar.ring_full[(n + 1) & 1], ((n + 1) >> 1) & 1, bar.abort_flag, status)))
+                        break;
+                    if (!(ok = mbar_wait(bar.p_read, n & 1, bar.abort_flag, status))) break;
+                    tc_fence_after();
+                    issue_s(n + 1);
                 }
+                // dK += dS^T Q
+                if (!(ok = mbar_wait(bar.ds_ready, n & 1, bar.abort_flag, status))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kBlockM / 16; ++kk)
+                    mma_ts_lh<idesc_ts>(tmem + kDK, tmem + kDP + bwd_kcol(kk),
+                                        static_cast<uint32_t>(dq_mn) + ring + ((kk * 16 * 128) >> 4), hi_mn,
+                                        (n > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&bar.ring_empty[st]);
             }
             mma_commit(bar.acc_done);
@@ -325,7 +363,8 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
         __syncwarp();
     } else {
         // ------------------------------------------------------------ element-wise
-        const int quarter = warp & 3;
+        const int quarter = warp & 3;                       // TMEM lane quarter
+        const int ch = warp >> 2;                           // query columns 64 ch .. 64 ch + 63
         const int jj = quarter * 32 + lane;                 // key row of the tile (TMEM lane)
         const int j = k0 + jj;                              // key index in the sequence
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
@@ -348,46 +387,104 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
             tc_fence_after();
             const float* l2 = lse_s + st * kBlockM;
             const float* dl = dlt_s + st * kBlockM;
-#pragma unroll 1
-            for (int c = 0; c < kBlockM / 32; ++c) {
-                uint32_t sr[32], dr[32];
-                tmem_ld32(tmem + lane_addr + kS + c * 32, sr);
-                tmem_ld32(tmem + lane_addr + kDP + c * 32, dr);
-                tmem_wait_ld();
-                uint32_t pk[16], dk16[16];
+            // every pair of this warp's keys and query columns visible?  Then the
+            // loops below skip the mask (every tile of a non-causal sequence but
+            // its ragged last one)
+            const int i0 = qt * kBlockM + ch * 64;
+            const bool full = __all_sync(0xffffffffu, i_span != 0u && i_base <= i0 &&
+                                                          i0 + 63 <= i_base + static_cast<int>(i_span));
+            // P^T = exp2(s * log2(e) / sqrt(D) - lse * log2(e)) on visible pairs, as
+            // bf16 at bwd_pcol(c); the second chunk's load is in flight while the
+            // first is computed
+            {
+                uint32_t sbuf[2][32];
+                tmem_ld32(tmem + lane_addr + kS + ch * 64, sbuf[0]);
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float pv[2], dsv[2];
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = 2 * ch + cc;
+                    tmem_wait_ld();
+                    if (cc == 0) tmem_ld32(tmem + lane_addr + kS + ch * 64 + 32, sbuf[1]);
+                    const uint32_t* sr = sbuf[cc];
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int col = c * 32 + e + u;
-                        const int i = qt * kBlockM + col;
-                        const bool vis = static_cast<unsigned>(i - i_base) <= i_span;
-                        const float pe = vis ? ex2_approx(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -l2[col]))
-                                             : 0.f;
-                        pv[u] = pe;
-                        dsv[u] = pe * (__uint_as_float(dr[e + u]) - dl[col]);
+                    for (int e = 0; e < 32; e += 4) {
+                        const float4 lv = *reinterpret_cast<const float4*>(l2 + c * 32 + e);
+                        const float lw[4] = {lv.x, lv.y, lv.z, lv.w};
+                        float pv[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float pe = ex2_approx(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -lw[u]));
+                            const int i = qt * kBlockM + c * 32 + e + u;
+                            pv[u] = (full || static_cast<unsigned>(i - i_base) <= i_span) ? pe : 0.f;
+                        }
+                        pk[e / 2] = pack_bf16x2(pv[0], pv[1]);
+                        pk[e / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
                     }
-                    pk[e / 2] = pack_bf16x2(pv[0], pv[1]);
-                    dk16[e / 2] = pack_bf16x2(dsv[0], dsv[1]);
+                    tmem_st16(tmem + lane_addr + kS + bwd_pcol(c), pk);
                 }
-                // P^T and dS^T over the S^T / dP^T columns this and earlier chunks have read
-                tmem_st16(tmem + lane_addr + kS + c * 16, pk);
-                tmem_st16(tmem + lane_addr + kDP + c * 16, dk16);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar.p_ready);
+            // dS^T = P^T (dP^T - Delta) from the stored bf16 P^T, as bf16 at
+            // kDP + bwd_pcol(c)
+            if (!(ok = mbar_wait_warp(bar.dp_full, n & 1, bar.abort_flag, status))) break;
+            tc_fence_after();
+            {
+                uint32_t dbuf[2][32], pbuf[2][16];
+                tmem_ld32(tmem + lane_addr + kDP + ch * 64, dbuf[0]);
+                tmem_ld16(tmem + lane_addr + kS + bwd_pcol(2 * ch), pbuf[0]);
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = 2 * ch + cc;
+                    tmem_wait_ld();
+                    if (cc == 0) {
+                        tmem_ld32(tmem + lane_addr + kDP + ch * 64 + 32, dbuf[1]);
+                        tmem_ld16(tmem + lane_addr + kS + bwd_pcol(c + 1), pbuf[1]);
+                    } else {
+                        // every P^T value of this warp is in registers: the next S^T may land
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar.p_read);
+                    }
+                    const uint32_t* dr = dbuf[cc];
+                    const uint32_t* pr = pbuf[cc];
+                    uint32_t dk16[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        const float4 dv4 = *reinterpret_cast<const float4*>(dl + c * 32 + e);
+                        const float dw[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+                        float ds[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint32_t w = pr[(e + u) / 2];
+                            const float pe = __uint_as_float(((e + u) & 1) ? (w & 0xFFFF0000u) : (w << 16));
+                            // masked pairs have P = 0 and stay exactly 0 (the Delta of a
+                            // row no key of this tile sees is never needed)
+                            ds[u] = pe != 0.f ? pe * (__uint_as_float(dr[e + u]) - dw[u]) : 0.f;
+                        }
+                        dk16[e / 2] = pack_bf16x2(ds[0], ds[1]);
+                        dk16[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+                    }
+                    tmem_st16(tmem + lane_addr + kDP + bwd_pcol(c), dk16);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar.ds_ready);
         }
         if (ok) ok = mbar_wait_warp(bar.acc_done, 0, bar.abort_flag, status);
         if (ok) {
             tc_fence_after();
+            // this warp's half of the D columns of its 32 key rows
             const bool valid = j < L_k;
-            uint8_t* base_v = p.dv + (static_cast<long long>(ck) + k0) * kv_pitch + hk * D * 2;
-            uint8_t* base_k = p.dk + (static_cast<long long>(ck) + k0) * kv_pitch + hk * D * 2;
-            bwd_store_rows<D>(tmem + lane_addr + kDV, 1.f, base_v, kv_pitch, jj, valid);
-            bwd_store_rows<D>(tmem + lane_addr + kDK, p.scale, base_k, kv_pitch, jj, valid);
+            const long long col = hk * D * 2 + ch * D;  // bytes
+            uint8_t* base_v = p.dv + (static_cast<long long>(ck) + k0) * kv_pitch + col;
+            uint8_t* base_k = p.dk + (static_cast<long long>(ck) + k0) * kv_pitch + col;
+            bwd_store_rows<D / 2>(tmem + lane_addr + kDV + ch * (D / 2), 1.f, base_v, kv_pitch, jj, valid);
+            bwd_store_rows<D / 2>(tmem + lane_addr + kDK + ch * (D / 2), p.scale, base_k, kv_pitch, jj, valid);
         }
     }
     bwd_teardown<D>(bar, tmem, warp);
@@ -469,31 +566,49 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
             const uint32_t hi_k = static_cast<uint32_t>(dq_ >> 32), hi_mn = static_cast<uint32_t>(dk_mn >> 32);
             bool ok = mbar_wait(bar.fixed_full, 0, bar.abort_flag, status);
             tc_fence_after();
-            for (int n = 0; n < n_steps && ok; ++n) {
-                const int st = n & 1;
-                if (!(ok = mbar_wait(&bar.ring_full[st], (n >> 1) & 1, bar.abort_flag, status))) break;
-                tc_fence_after();
-                const uint32_t ring = (st * L::kTile) >> 4;
-                // S = Q K^T and dP = dout V^T (K-major operands, K = D)
+            // S = Q K^T for step m (K of ring stage m & 1, K-major operands, K = D)
+            auto issue_s = [&](int m) {
+                const uint32_t ring = ((m & 1) * L::kTile) >> 4;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * T::kChunkBytes + (kk & 3) * 32) >> 4;
                     mma_ss_lh<idesc_ss>(tmem + kS, static_cast<uint32_t>(dq_) + off, hi_k,
                                         static_cast<uint32_t>(dk_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
                 }
+                mma_commit(bar.s_full);
+            };
+            // Order per step n: dP(n), S(n+1) once the element-wise warps have read
+            // S(n), dQ(n) once dS(n) is stored.  The next S so runs while dS is
+            // formed; dP(n+1) overwrites dS(n) and follows dQ(n).
+            if (ok && n_steps > 0) {
+                ok = mbar_wait(&bar.ring_full[0], 0, bar.abort_flag, status);
+                tc_fence_after();
+                if (ok) issue_s(0);
+            }
+            for (int n = 0; n < n_steps && ok; ++n) {
+                const int st = n & 1;
+                const uint32_t ring = (st * L::kTile) >> 4;
+                // dP = dout V^T (K-major operands, K = D)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * T::kChunkBytes + (kk & 3) * 32) >> 4;
                     mma_ss_lh<idesc_ss>(tmem + kDP, static_cast<uint32_t>(dd_) + off, hi_k,
                                         static_cast<uint32_t>(dv_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(bar.s_full);
+                mma_commit(bar.dp_full);
+                if (n + 1 < n_steps) {
+                    if (!(ok = mbar_wait(&bar.ring_full[(n + 1) & 1], ((n + 1) >> 1) & 1, bar.abort_flag, status)))
+                        break;
+                    if (!(ok = mbar_wait(bar.p_read, n & 1, bar.abort_flag, status))) break;
+                    tc_fence_after();
+                    issue_s(n + 1);
+                }
                 if (!(ok = mbar_wait(bar.p_ready, n & 1, bar.abort_flag, status))) break;
                 tc_fence_after();
                 // dQ += dS K (A from tensor memory, B = K MN-major, K = 128 keys)
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    mma_ts_lh<idesc_ts>(tmem + kDQ, tmem + kDP + kk * 8,
+                    mma_ts_lh<idesc_ts>(tmem + kDQ, tmem + kDP + bwd_kcol(kk),
                                         static_cast<uint32_t>(dk_mn) + ring + ((kk * 16 * 128) >> 4), hi_mn,
                                         (n > 0 || kk > 0) ? 1u : 0u);
                 }
@@ -504,7 +619,8 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
         __syncwarp();
     } else {
         // ------------------------------------------------------------ element-wise
-        const int quarter = warp & 3;
+        const int quarter = warp & 3;        // TMEM lane quarter
+        const int ch = warp >> 2;            // key columns 64 ch .. 64 ch + 63
         const int ii = quarter * 32 + lane;  // query row of the tile (TMEM lane)
         const int i = q0 + ii;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
@@ -512,9 +628,25 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
         float l2 = 0.f, dl = 0.f;
         int lo = 0, hi = -1;
         if (row_valid) {
-            const float l = p.lse[static_cast<size_t>(cq + i) * p.H + h];
+            const size_t row = static_cast<size_t>(cq + i) * p.H + h;
+            const float l = p.lse[row];
             l2 = l == -INFINITY ? 0.f : l * 1.4426950408889634f;
-            dl = p.delta[static_cast<size_t>(cq + i) * p.H + h];
+            // Delta_i = dout_i . out_i, kept here and stored for the dK/dV kernel
+            const uint4* o4 = reinterpret_cast<const uint4*>(p.out + row * (D * 2));
+            const uint4* g4 = reinterpret_cast<const uint4*>(p.dout + row * (D * 2));
+            float acc = 0.f;
+#pragma unroll 4
+            for (int c = 0; c < D / 8; ++c) {
+                const uint4 a = o4[c], g = g4[c];
+                const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    acc = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(gv[e] << 16), acc);
+                    acc = fmaf(__uint_as_float(av[e] & 0xFFFF0000u), __uint_as_float(gv[e] & 0xFFFF0000u), acc);
+                }
+            }
+            dl = acc;
+            if (ch == 0) p.rowinfo[h * p.rows_cap + cq + i] = make_float2(l2, acc);
             row_key_interval(i, L_q, L_k, p.causal != 0, p.window, lo, hi);
         }
         const unsigned span = hi >= lo ? static_cast<unsigned>(hi - lo) : 0u;
@@ -524,27 +656,48 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
             const int kt = kt_lo + n;
             if (!(ok = mbar_wait_warp(bar.s_full, n & 1, bar.abort_flag, status))) break;
             tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < kBlockN / 32; ++c) {
-                uint32_t sr[32], dr[32];
-                tmem_ld32(tmem + lane_addr + kS + c * 32, sr);
-                tmem_ld32(tmem + lane_addr + kDP + c * 32, dr);
+            // all of this warp's rows see every key of its columns?  (skip the mask)
+            const int k0c = kt * kBlockN + ch * 64;
+            const bool full = __all_sync(0xffffffffu, hi >= lo && lo <= k0c && k0c + 63 <= hi);
+            // P = exp2(s * log2(e) / sqrt(D) - lse * log2(e)) on visible pairs, in
+            // registers; then S may be overwritten by the next step's product
+            float pv[64];
+            {
+                uint32_t sbuf[2][32];
+                tmem_ld32(tmem + lane_addr + kS + ch * 64, sbuf[0]);
+                tmem_ld32(tmem + lane_addr + kS + ch * 64 + 32, sbuf[1]);
                 tmem_wait_ld();
-                uint32_t dk16[16];
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar.p_read);
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float dsv[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int jkey = kt * kBlockN + c * 32 + e + u;
-                        const bool vis = static_cast<unsigned>(jkey - base) <= span;
-                        const float pe = vis ? ex2_approx(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -l2)) : 0.f;
-                        dsv[u] = pe * (__uint_as_float(dr[e + u]) - dl);
-                    }
-                    dk16[e / 2] = pack_bf16x2(dsv[0], dsv[1]);
+                for (int e = 0; e < 64; ++e) {
+                    const int jkey = k0c + e;
+                    const bool vis = full || static_cast<unsigned>(jkey - base) <= span;
+                    const float pe = ex2_approx(fmaf(__uint_as_float(sbuf[e >> 5][e & 31]), p.scale_log2, -l2));
+                    pv[e] = vis ? pe : 0.f;
                 }
-                // dS over the dP columns this and earlier chunks have read
-                tmem_st16(tmem + lane_addr + kDP + c * 16, dk16);
+            }
+            // dS = P (dP - Delta) as bf16 at kDP + bwd_pcol(c), over dP columns read
+            if (!(ok = mbar_wait_warp(bar.dp_full, n & 1, bar.abort_flag, status))) break;
+            tc_fence_after();
+            {
+                uint32_t dbuf[2][32];
+                tmem_ld32(tmem + lane_addr + kDP + ch * 64, dbuf[0]);
+                tmem_ld32(tmem + lane_addr + kDP + ch * 64 + 32, dbuf[1]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint32_t dk16[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const float* pp = pv + cc * 32 + e;
+                        const float d0 = pp[0] != 0.f ? pp[0] * (__uint_as_float(dbuf[cc][e]) - dl) : 0.f;
+                        const float d1 = pp[1] != 0.f ? pp[1] * (__uint_as_float(dbuf[cc][e + 1]) - dl) : 0.f;
+                        dk16[e / 2] = pack_bf16x2(d0, d1);
+                    }
+                    tmem_st16(tmem + lane_addr + kDP + bwd_pcol(2 * ch + cc), dk16);
+                }
             }
             tmem_wait_st();
             tc_fence_before();
@@ -554,8 +707,10 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
         if (ok) ok = mbar_wait_warp(bar.acc_done, 0, bar.abort_flag, status);
         if (ok) {
             tc_fence_after();
-            uint8_t* base_q = p.dq + (static_cast<long long>(cq) + q0) * q_pitch + h * D * 2;
-            bwd_store_rows<D>(tmem + lane_addr + kDQ, p.scale, base_q, q_pitch, ii, row_valid);
+            // this warp's half of the D columns of its 32 query rows
+            uint8_t* base_q = p.dq + (static_cast<long long>(cq) + q0) * q_pitch + h * D * 2 + ch * D;
+            bwd_store_rows<D / 2>(tmem + lane_addr + kDQ + ch * (D / 2), p.scale, base_q, q_pitch, ii,
+                                  row_valid);
         }
     }
     bwd_teardown<D>(bar, tmem, warp);

@@ -426,8 +426,8 @@ int forward(const Args& a, int path, int split_keys, cudaStream_t stream) {
 }
 
 // ---------------------------------------------------------------------------
-// Backward pass: Delta = rowsum(dout * out), then dK/dV per key tile and dQ
-// per query tile (backward_sm100.cuh).
+// Backward pass: dQ per query tile (which also forms Delta = rowsum(dout *
+// out)), then dK/dV per key tile (backward_sm100.cuh).
 
 struct BwdArgs {
     Args fwd;  // q, k, v, cu_seqlens, sizes, masks; out = the forward output, lse its logsumexp
@@ -467,8 +467,8 @@ int run_backward(const BwdArgs& g, cudaStream_t stream) {
         (rc = make_tile_map(&maps.k8, a.k, cols_k, rows_k, 8)) != VA_OK ||
         (rc = make_tile_map(&maps.v8, a.v, cols_k, rows_k, 8)) != VA_OK)
         return rc;
-    float* delta = nullptr;
-    VA_CUDA(ws_alloc(reinterpret_cast<void**>(&delta), static_cast<size_t>(rows_q) * a.H * sizeof(float),
+    float2* rowinfo = nullptr;
+    VA_CUDA(ws_alloc(reinterpret_cast<void**>(&rowinfo), static_cast<size_t>(rows_q) * a.H * sizeof(float2),
                      stream));
     va::BwdParams p;
     p.cu_q = a.cu_q;
@@ -484,29 +484,28 @@ int run_backward(const BwdArgs& g, cudaStream_t stream) {
     p.dout = static_cast<const uint8_t*>(g.dout);
     p.out = static_cast<const uint8_t*>(a.out);
     p.lse = a.lse;
-    p.delta = delta;
+    p.rowinfo = rowinfo;
+    p.rows_cap = rows_q;
     p.dq = static_cast<uint8_t*>(g.dq);
     p.dk = static_cast<uint8_t*>(g.dk);
     p.dv = static_cast<uint8_t*>(g.dv);
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(a.D)));
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)));
-    const long long delta_rows = rows_q * a.H;
-    const unsigned delta_blocks = static_cast<unsigned>((delta_rows + 7) / 8);
     const dim3 grid_kv(static_cast<unsigned>((std::max(a.max_k, 1) + va::kBlockN - 1) / va::kBlockN),
                        static_cast<unsigned>(a.H_kv), static_cast<unsigned>(a.batch));
     const dim3 grid_q(static_cast<unsigned>((std::max(a.max_q, 1) + va::kBlockM - 1) / va::kBlockM),
                       static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch));
+    // dQ first: it forms Delta for every query row that sees a key, which the
+    // dK/dV kernel reads
     if (a.D == 64) {
-        va::bwd_delta_kernel<64><<<delta_blocks, 256, 0, stream>>>(p);
-        va::bwd_dkdv_kernel<64><<<grid_kv, va::kBwdThreads, va::BwdSmem<64>::kAlloc, stream>>>(maps, p);
         va::bwd_dq_kernel<64><<<grid_q, va::kBwdThreads, va::BwdSmem<64>::kAlloc, stream>>>(maps, p);
+        va::bwd_dkdv_kernel<64><<<grid_kv, va::kBwdThreads, va::BwdSmem<64>::kAlloc, stream>>>(maps, p);
     } else {
-        va::bwd_delta_kernel<128><<<delta_blocks, 256, 0, stream>>>(p);
-        va::bwd_dkdv_kernel<128><<<grid_kv, va::kBwdThreads, va::BwdSmem<128>::kAlloc, stream>>>(maps, p);
         va::bwd_dq_kernel<128><<<grid_q, va::kBwdThreads, va::BwdSmem<128>::kAlloc, stream>>>(maps, p);
+        va::bwd_dkdv_kernel<128><<<grid_kv, va::kBwdThreads, va::BwdSmem<128>::kAlloc, stream>>>(maps, p);
     }
     cudaError_t le = cudaGetLastError();
-    cudaFreeAsync(delta, stream);
+    cudaFreeAsync(rowinfo, stream);
     if (le != cudaSuccess) return cuda_fail(le, "backward launch");
     return VA_OK;
 }
