@@ -317,6 +317,18 @@ def run_profile_target(args, local):
     ck = torch.tensor(wl.cu_k, dtype=torch.int32, device=dev)
     out = torch.empty_like(dq)
     lse = torch.empty(wl.total_q, wl.H, dtype=torch.float32, device=dev)
+    if args.only == "bwd":
+        binding.varlen_attention_fwd(dq, dk, dv, cq, ck, wl.batch, wl.H, wl.H_kv, wl.max_seqlen_q,
+                                     wl.max_seqlen_k, wl.D, wl.causal, wl.window, out=out, lse=lse)
+        gen = torch.Generator().manual_seed(workloads.WORKLOAD_SEEDS[args.workload] + 7)
+        ddo = torch.randn(wl.total_q, wl.H, wl.D, generator=gen).to(torch.bfloat16).to(dev)
+        for _ in range(args.warmup + args.steps):
+            binding.varlen_attention_bwd(ddo, dq, dk, dv, out, lse, cq, ck, wl.batch, wl.H, wl.H_kv,
+                                         wl.max_seqlen_q, wl.max_seqlen_k, wl.D, wl.causal, wl.window)
+        torch.cuda.synchronize()
+        if binding.device_status() != 0:
+            raise SystemExit("device status word raised")
+        return
     for _ in range(args.warmup + args.steps):
         binding.varlen_attention_fwd(dq, dk, dv, cq, ck, wl.batch, wl.H, wl.H_kv, wl.max_seqlen_q,
                                      wl.max_seqlen_k, wl.D, wl.causal, wl.window, out=out, lse=lse)
@@ -532,7 +544,7 @@ def main():
     ap.add_argument("--no-clock-sampler", action="store_true")
     ap.add_argument("--scale", type=float, default=1.0,
                     help="shrink every sequence length (profiling captures of a small case)")
-    ap.add_argument("--only", choices=["all", "prefill", "fp8", "decode"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "fp8", "bwd", "decode"], default="all",
                     help="profiling: run only one half of the step (no JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
