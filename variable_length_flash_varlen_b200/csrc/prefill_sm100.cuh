@@ -240,6 +240,39 @@ __device__ __forceinline__ void store_row_zero(const PrefillParams& p, size_t ou
     p.lse[out_row] = -INFINITY;
 }
 
+// Packed pairs of f32 in one 64-bit register (lo, hi): one instruction of the
+// f32x2 forms does two lanes' worth of FMA-pipe work, which halves the issue
+// slots of the element-wise softmax arithmetic.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+// max of three (one instruction)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 template <int D, class E>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams p) {
@@ -579,16 +612,19 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                     for (int c = 0; c < kBlockN; ++c)
                         s[c] = (static_cast<unsigned>(c - c_lo) <= span) ? s[c] : -INFINITY;
                 }
-                // row max as a tree (short dependency chains)
+                // row max as a tree of three-input maxima (eight short chains)
+                static_assert(kBlockN == 128, "the max tree covers 128 columns");
                 float mv[8];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) mv[c] = s[c];
+                for (int e = 0; e < 8; ++e) mv[e] = max3f(s[e], s[8 + e], s[16 + e]);
 #pragma unroll
-                for (int c = 8; c < kBlockN; c += 8)
+                for (int c = 24; c < 120; c += 16)
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) mv[e] = fmaxf(mv[e], s[c + e]);
-                const float mx = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
-                                       fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
+                    for (int e = 0; e < 8; ++e) mv[e] = max3f(mv[e], s[c + e], s[c + 8 + e]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mv[e] = fmaxf(mv[e], s[120 + e]);
+                const float mx = max3f(max3f(mv[0], mv[1], mv[2]), max3f(mv[3], mv[4], mv[5]),
+                                       fmaxf(mv[6], mv[7]));
                 const float m_tile = mx * p.scale_log2;  // -inf stays -inf
                 const float m_cand = fmaxf(m_ref, m_tile);
                 const bool want = first_tile || (m_cand > m_ref + kRescaleThreshold);
@@ -603,7 +639,10 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                 // pairs or E4M3 quadruples), 64 keys at a time; the first 64 are handed over on their own so
                 // their PV starts while the second half is computed.  S_x's previous P
                 // was consumed by the PV issued before this QK.
-                float sums[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                // (pairs of columns through the packed f32x2 FMA and add)
+                const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+                const uint64_t neg2 = f2_pack(-m_sub, -m_sub);
+                uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};  // eight partial sums, as pairs
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     if constexpr (E::kFp8) {
@@ -611,11 +650,15 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                         uint32_t pk[16];
 #pragma unroll
                         for (int c = 0; c < 64; c += 4) {
-                            const float p0 = ex2_approx(fmaf(s[half * 64 + c], p.scale_log2, -m_sub));
-                            const float p1 = ex2_approx(fmaf(s[half * 64 + c + 1], p.scale_log2, -m_sub));
-                            const float p2 = ex2_approx(fmaf(s[half * 64 + c + 2], p.scale_log2, -m_sub));
-                            const float p3 = ex2_approx(fmaf(s[half * 64 + c + 3], p.scale_log2, -m_sub));
-                            sums[(c >> 2) & 7] += (p0 + p1) + (p2 + p3);
+                            float x0, x1, x2, x3;
+                            f2_unpack(f2_fma(f2_pack(s[half * 64 + c], s[half * 64 + c + 1]), scale2, neg2),
+                                      x0, x1);
+                            f2_unpack(f2_fma(f2_pack(s[half * 64 + c + 2], s[half * 64 + c + 3]), scale2,
+                                             neg2),
+                                      x2, x3);
+                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+                            sum2[(c >> 2) & 3] = f2_add(sum2[(c >> 2) & 3], f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
                             pk[c / 4] = pack_e4m3x4(p0, p1, p2, p3);
                         }
                         tmem_st16(sbase + half * 16, pk);
@@ -623,9 +666,11 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                         uint32_t pk[32];
 #pragma unroll
                         for (int c = 0; c < 64; c += 2) {
-                            const float p0 = ex2_approx(fmaf(s[half * 64 + c], p.scale_log2, -m_sub));
-                            const float p1 = ex2_approx(fmaf(s[half * 64 + c + 1], p.scale_log2, -m_sub));
-                            sums[(c >> 1) & 7] += p0 + p1;
+                            float x0, x1;
+                            f2_unpack(f2_fma(f2_pack(s[half * 64 + c], s[half * 64 + c + 1]), scale2, neg2),
+                                      x0, x1);
+                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            sum2[(c >> 1) & 3] = f2_add(sum2[(c >> 1) & 3], f2_pack(p0, p1));
                             pk[c / 2] = pack_bf16x2(p0, p1);
                         }
                         tmem_st32(sbase + half * 32, pk);
@@ -652,6 +697,9 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                         if (lane == 0) mbar_arrive(&p_half[x]);
                     }
                 }
+                float sums[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) f2_unpack(sum2[e], sums[2 * e], sums[2 * e + 1]);
                 l = l * alpha + (((sums[0] + sums[1]) + (sums[2] + sums[3])) +
                                  ((sums[4] + sums[5]) + (sums[6] + sums[7])));
                 tmem_wait_st();
