@@ -57,7 +57,8 @@ def load_peaks():
 # included), so a recorded traffic figure goes stale only when its own kernel
 # changes.
 KERNEL_SOURCES = {
-    "prefill_fwd_kernel": ("prefill_sm100.cuh", "schedule.cuh", "ptx.cuh", "status.cuh", "varlen_attn.cu"),
+    "prefill_fwd_kernel": ("prefill_sm100.cuh", "f32x2.cuh", "schedule.cuh", "ptx.cuh", "status.cuh",
+                           "varlen_attn.cu"),
     "decode_stream_kernel": ("decode.cuh", "schedule.cuh", "ptx.cuh", "status.cuh", "varlen_attn.cu"),
 }
 

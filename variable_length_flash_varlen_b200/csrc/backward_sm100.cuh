@@ -259,8 +259,9 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
             if (!(ok = mbar_wait_warp(&bar.ring_empty[st], ((n >> 1) & 1) ^ 1, bar.abort_flag, status)))
                 break;
             {
-                // the tile's 128 rows of {lse * log2(e), Delta}: four loads per lane in
-                // flight at once (rows past the sequence are masked: any finite value)
+                // the tile's 128 rows of {lse * log2(e), Delta}, staged negated (the
+                // element-wise warps add them): four loads per lane in flight at once
+                // (rows past the sequence are masked: any finite value)
                 const float2* src = p.rowinfo + h * p.rows_cap + cq + qt * kBlockM;
                 float2 ri[kBlockM / 32];
 #pragma unroll
@@ -270,8 +271,8 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                 }
 #pragma unroll
                 for (int u = 0; u < kBlockM / 32; ++u) {
-                    lse_s[st * kBlockM + lane + 32 * u] = ri[u].x;
-                    dlt_s[st * kBlockM + lane + 32 * u] = ri[u].y;
+                    lse_s[st * kBlockM + lane + 32 * u] = -ri[u].x;
+                    dlt_s[st * kBlockM + lane + 32 * u] = -ri[u].y;
                 }
             }
             __syncwarp();
@@ -375,6 +376,7 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
         if (j >= L_k) i_hi = -1;
         const unsigned i_span = i_hi >= i_lo ? static_cast<unsigned>(i_hi - i_lo) : 0u;
         const int i_base = i_hi >= i_lo ? i_lo : (1 << 30);
+        const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
         bool ok = true;
         for (int n = 0; n < n_steps; ++n) {
             const int st = n & 1;
@@ -385,8 +387,8 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
             // warp waited for it before the products this wait observed)
             if (!(ok = mbar_wait_warp(&bar.ring_full[st], (n >> 1) & 1, bar.abort_flag, status))) break;
             tc_fence_after();
-            const float* l2 = lse_s + st * kBlockM;
-            const float* dl = dlt_s + st * kBlockM;
+            const float* nl2 = lse_s + st * kBlockM;  // -lse * log2(e) per query column
+            const float* ndl = dlt_s + st * kBlockM;  // -Delta per query column
             // every pair of this warp's keys and query columns visible?  Then the
             // loops below skip the mask (every tile of a non-causal sequence but
             // its ragged last one)
@@ -405,21 +407,31 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                     tmem_wait_ld();
                     if (cc == 0) tmem_ld32(tmem + lane_addr + kS + ch * 64 + 32, sbuf[1]);
                     const uint32_t* sr = sbuf[cc];
-                    uint32_t pk[16];
+                    // scale and shift as packed pairs, then the mask (only on tiles
+                    // where some pair of this warp is not visible)
+                    float pv[32];
 #pragma unroll
                     for (int e = 0; e < 32; e += 4) {
-                        const float4 lv = *reinterpret_cast<const float4*>(l2 + c * 32 + e);
-                        const float lw[4] = {lv.x, lv.y, lv.z, lv.w};
-                        float pv[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const float pe = ex2_approx(fmaf(__uint_as_float(sr[e + u]), p.scale_log2, -lw[u]));
-                            const int i = qt * kBlockM + c * 32 + e + u;
-                            pv[u] = (full || static_cast<unsigned>(i - i_base) <= i_span) ? pe : 0.f;
-                        }
-                        pk[e / 2] = pack_bf16x2(pv[0], pv[1]);
-                        pk[e / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+                        const float4 nl = *reinterpret_cast<const float4*>(nl2 + c * 32 + e);
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), scale2,
+                                         f2_pack(nl.x, nl.y)),
+                                  pv[e], pv[e + 1]);
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3])), scale2,
+                                         f2_pack(nl.z, nl.w)),
+                                  pv[e + 2], pv[e + 3]);
                     }
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) pv[e] = ex2_approx(pv[e]);
+                    if (!full) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int i = qt * kBlockM + c * 32 + e;
+                            pv[e] = static_cast<unsigned>(i - i_base) <= i_span ? pv[e] : 0.f;
+                        }
+                    }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) pk[e / 2] = pack_bf16x2(pv[e], pv[e + 1]);
                     tmem_st16(tmem + lane_addr + kS + bwd_pcol(c), pk);
                 }
             }
@@ -450,19 +462,21 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                     }
                     const uint32_t* dr = dbuf[cc];
                     const uint32_t* pr = pbuf[cc];
+                    // dS = P (dP - Delta) on packed pairs; a masked pair has P = 0 and a
+                    // finite dP - Delta (rows past the sequence stage Delta = 0), so it
+                    // stays 0
                     uint32_t dk16[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 4) {
-                        const float4 dv4 = *reinterpret_cast<const float4*>(dl + c * 32 + e);
-                        const float dw[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+                        const float4 nd = *reinterpret_cast<const float4*>(ndl + c * 32 + e);
                         float ds[4];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
+                        for (int u = 0; u < 4; u += 2) {
                             const uint32_t w = pr[(e + u) / 2];
-                            const float pe = __uint_as_float(((e + u) & 1) ? (w & 0xFFFF0000u) : (w << 16));
-                            // masked pairs have P = 0 and stay exactly 0 (the Delta of a
-                            // row no key of this tile sees is never needed)
-                            ds[u] = pe != 0.f ? pe * (__uint_as_float(dr[e + u]) - dw[u]) : 0.f;
+                            const uint64_t p2 = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+                            const uint64_t d2 = f2_add(f2_pack(__uint_as_float(dr[e + u]), __uint_as_float(dr[e + u + 1])),
+                                                       u == 0 ? f2_pack(nd.x, nd.y) : f2_pack(nd.z, nd.w));
+                            f2_unpack(f2_mul(p2, d2), ds[u], ds[u + 1]);
                         }
                         dk16[e / 2] = pack_bf16x2(ds[0], ds[1]);
                         dk16[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
@@ -651,6 +665,8 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
         }
         const unsigned span = hi >= lo ? static_cast<unsigned>(hi - lo) : 0u;
         const int base = hi >= lo ? lo : (1 << 30);
+        const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nl2 = f2_pack(-l2, -l2), ndl2 = f2_pack(-dl, -dl);
         bool ok = true;
         for (int n = 0; n < n_steps; ++n) {
             const int kt = kt_lo + n;
@@ -671,11 +687,17 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar.p_read);
 #pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                    const int jkey = k0c + e;
-                    const bool vis = full || static_cast<unsigned>(jkey - base) <= span;
-                    const float pe = ex2_approx(fmaf(__uint_as_float(sbuf[e >> 5][e & 31]), p.scale_log2, -l2));
-                    pv[e] = vis ? pe : 0.f;
+                for (int e = 0; e < 64; e += 2)
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sbuf[e >> 5][e & 31]),
+                                             __uint_as_float(sbuf[e >> 5][(e & 31) + 1])),
+                                     scale2, nl2),
+                              pv[e], pv[e + 1]);
+#pragma unroll
+                for (int e = 0; e < 64; ++e) pv[e] = ex2_approx(pv[e]);
+                if (!full) {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e)
+                        pv[e] = static_cast<unsigned>(k0c + e - base) <= span ? pv[e] : 0.f;
                 }
             }
             // dS = P (dP - Delta) as bf16 at kDP + bwd_pcol(c), over dP columns read
@@ -691,9 +713,12 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                     uint32_t dk16[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        const float* pp = pv + cc * 32 + e;
-                        const float d0 = pp[0] != 0.f ? pp[0] * (__uint_as_float(dbuf[cc][e]) - dl) : 0.f;
-                        const float d1 = pp[1] != 0.f ? pp[1] * (__uint_as_float(dbuf[cc][e + 1]) - dl) : 0.f;
+                        // a masked pair has P = 0 and a finite dP - Delta: it stays 0
+                        float d0, d1;
+                        f2_unpack(f2_mul(f2_pack(pv[cc * 32 + e], pv[cc * 32 + e + 1]),
+                                         f2_add(f2_pack(__uint_as_float(dbuf[cc][e]), __uint_as_float(dbuf[cc][e + 1])),
+                                                ndl2)),
+                                  d0, d1);
                         dk16[e / 2] = pack_bf16x2(d0, d1);
                     }
                     tmem_st16(tmem + lane_addr + kDP + bwd_pcol(2 * ch + cc), dk16);

@@ -37,6 +37,7 @@
 
 #include <cuda_bf16.h>
 
+#include "f32x2.cuh"
 #include "ptx.cuh"
 #include "schedule.cuh"
 #include "status.cuh"
@@ -238,39 +239,6 @@ __device__ __forceinline__ void store_row_zero(const PrefillParams& p, size_t ou
 #pragma unroll
     for (int c = 0; c < D * E::kBytes / 16; ++c) o4[c] = make_uint4(0u, 0u, 0u, 0u);
     p.lse[out_row] = -INFINITY;
-}
-
-// Packed pairs of f32 in one 64-bit register (lo, hi): one instruction of the
-// f32x2 forms does two lanes' worth of FMA-pipe work, which halves the issue
-// slots of the element-wise softmax arithmetic.
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t r;
-    asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-// max of three (one instruction)
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
 }
 
 template <int D, class E>
