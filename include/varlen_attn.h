@@ -176,7 +176,13 @@ int varlen_attention_fwd_ex(const void* q, const void* k, const void* v,
  * gives asynchronous copies; pageable memory works but is staged by CUDA).
  * Copies inputs to the device, runs varlen_attention_fwd on `stream`, copies
  * out and lse back and synchronises `stream` before returning.  Device
- * buffers are allocated and freed stream-ordered inside the call.
+ * buffers are allocated and freed stream-ordered inside the call.  Once the
+ * inputs reach 8 MiB the batch is split into up to four chunks of whole
+ * sequences (balanced by query tokens) and pipelined: each chunk's kernels
+ * run on `stream` while the next chunk is copied in and the previous one
+ * copied out on two library-owned copy streams (created on the first such
+ * call per device); the results are bit-identical to one launch over the
+ * whole batch.
  */
 int varlen_attention_fwd_host(const void* q, const void* k, const void* v,
                               const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,

@@ -128,6 +128,25 @@ def test_host_buffer_entry_matches_device_entry():
     assert torch.equal(out_h, out_d.cpu()) and torch.equal(lse_h, lse_d.cpu())
 
 
+def test_host_buffer_entry_pipelined_chunks_match_device_entry():
+    # inputs above the pipelining threshold: the host entry splits the batch
+    # into chunks of whole sequences, each copied in, computed and copied out
+    # on its own; every sequence's result is independent of the launch that
+    # computes it, so the results are bit-identical to the device entry's
+    wl = workloads.named("mha_noncausal", scale=0.5)
+    q, k, v = workloads.make_qkv(wl)
+    assert (q.numel() + k.numel() + v.numel()) * 2 >= 8 << 20
+    out_d, lse_d = run_gpu(wl, q, k, v)
+    out_h = torch.full_like(q, float("nan")).pin_memory()
+    lse_h = torch.full((wl.total_q, wl.H), float("nan"), dtype=torch.float32).pin_memory()
+    cq = torch.tensor(wl.cu_q, dtype=torch.int32)
+    ck = torch.tensor(wl.cu_k, dtype=torch.int32)
+    binding.varlen_attention_fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), cq, ck,
+                                      wl.batch, wl.H, wl.H_kv, wl.max_seqlen_q, wl.max_seqlen_k,
+                                      wl.D, wl.causal, wl.window, out_h, lse_h)
+    assert torch.equal(out_h, out_d.cpu()) and torch.equal(lse_h, lse_d.cpu())
+
+
 # --- decode path -------------------------------------------------------------------
 
 @pytest.mark.parametrize("split_keys", [32, 100, 448, 1024, 5000])

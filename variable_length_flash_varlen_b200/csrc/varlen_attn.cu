@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "backward_sm100.cuh"
 #include "decode.cuh"
@@ -60,6 +61,10 @@ int cuda_fail(cudaError_t e, const char* what) {
     } while (0)
 
 constexpr int kMaxDevices = 64;
+// Host-buffer entry point: up to this many pipelined chunks, once the inputs
+// reach this size.
+constexpr int kHostChunks = 4;
+constexpr size_t kHostChunkMinBytes = size_t(8) << 20;
 
 struct DeviceInfo {
     bool ready = false;
@@ -68,6 +73,8 @@ struct DeviceInfo {
     // unlimited, so a synchronisation does not hand its memory back to the OS
     // and the next call does not pay for mapping it again.
     cudaMemPool_t pool = nullptr;
+    // Copy streams of the host-buffer entry point (created on first use).
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -706,42 +713,128 @@ int varlen_attention_fwd_host(const void* q, const void* k, const void* v,
     if ((rc = device_setup(dev, info)) != VA_OK) return rc;
     const long long T_q = cu_seqlens_q[batch], T_k = cu_seqlens_k[batch];
     if (T_q < 0 || T_k < 0) return fail(VA_ERR_INVALID_ARG, "negative total length");
-    const size_t qb = static_cast<size_t>(T_q) * num_heads * head_dim * 2;
-    const size_t kb = static_cast<size_t>(T_k) * num_kv_heads * head_dim * 2;
-    const size_t cb = static_cast<size_t>(batch + 1) * 4;
-    const size_t ob = qb, lb = static_cast<size_t>(T_q) * num_heads * 4;
-    auto up16 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-    const size_t total = up16(qb) + 2 * up16(kb) + 2 * up16(cb) + up16(ob) + up16(lb);
+    const size_t q_row = static_cast<size_t>(num_heads) * head_dim * 2;
+    const size_t k_row = static_cast<size_t>(num_kv_heads) * head_dim * 2;
+    const size_t l_row = static_cast<size_t>(num_heads) * 4;
+    const size_t qb = static_cast<size_t>(T_q) * q_row, kb = static_cast<size_t>(T_k) * k_row;
+    const size_t ob = qb, lb = static_cast<size_t>(T_q) * l_row;
+
+    // Chunks of whole sequences, balanced by query tokens: chunk i's kernels
+    // run while chunk i + 1 is copied in and chunk i - 1 is copied out (the
+    // two directions on separate streams and copy engines).  Each sequence's
+    // result does not depend on which chunk or launch computes it.
+    std::vector<int> bounds{0};
+    const int n_want = (qb + 2 * kb >= kHostChunkMinBytes) ? std::min(kHostChunks, batch) : 1;
+    for (int c = 1; c < n_want; ++c) {
+        const long long target = T_q * c / n_want;
+        int b = bounds.back() + 1;
+        while (b < batch && cu_seqlens_q[b] < target) ++b;
+        if (b < batch) bounds.push_back(b);
+    }
+    bounds.push_back(batch);
+    const int n = static_cast<int>(bounds.size()) - 1;
+    // per chunk, cu_seqlens rebased to its first sequence (chunk c's arrays
+    // start at entry bounds[c] + c)
+    std::vector<int32_t> cu_h(2 * static_cast<size_t>(batch + n));
+    for (int c = 0; c < n; ++c)
+        for (int b = bounds[c]; b <= bounds[c + 1]; ++b) {
+            cu_h[b + c] = cu_seqlens_q[b] - cu_seqlens_q[bounds[c]];
+            cu_h[batch + n + b + c] = cu_seqlens_k[b] - cu_seqlens_k[bounds[c]];
+        }
+    const size_t cb = cu_h.size() * sizeof(int32_t);
+
+    auto up256 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    const size_t total = up256(qb) + 2 * up256(kb) + up256(cb) + up256(ob) + up256(lb);
+    cudaStream_t s_in = stream, s_out = stream;
+    if (n > 1) {
+        std::lock_guard<std::mutex> lock(g_dev_mu);
+        if (!info->copy_in) VA_CUDA(cudaStreamCreateWithFlags(&info->copy_in, cudaStreamNonBlocking));
+        if (!info->copy_out) VA_CUDA(cudaStreamCreateWithFlags(&info->copy_out, cudaStreamNonBlocking));
+        s_in = info->copy_in;
+        s_out = info->copy_out;
+    }
     char* ws = nullptr;
     VA_CUDA(ws_alloc(reinterpret_cast<void**>(&ws), total, stream));
     char* p = ws;
-    void* dq = p; p += up16(qb);
-    void* dk = p; p += up16(kb);
-    void* dv = p; p += up16(kb);
-    int32_t* dcq = reinterpret_cast<int32_t*>(p); p += up16(cb);
-    int32_t* dck = reinterpret_cast<int32_t*>(p); p += up16(cb);
-    void* dout = p; p += up16(ob);
+    char* dq = p; p += up256(qb);
+    char* dk = p; p += up256(kb);
+    char* dv = p; p += up256(kb);
+    int32_t* dcu = reinterpret_cast<int32_t*>(p); p += up256(cb);
+    char* dout = p; p += up256(ob);
     float* dlse = reinterpret_cast<float*>(p);
+
+    // events: [0] workspace ready, [1 .. n] chunk c copied in, [n + 1 .. 2n]
+    // chunk c computed, [2n + 1] / [2n + 2] the copy streams drained
+    std::vector<cudaEvent_t> ev;
     cudaError_t e = cudaSuccess;
-    if (qb) e = cudaMemcpyAsync(dq, q, qb, cudaMemcpyHostToDevice, stream);
-    if (e == cudaSuccess && kb) e = cudaMemcpyAsync(dk, k, kb, cudaMemcpyHostToDevice, stream);
-    if (e == cudaSuccess && kb) e = cudaMemcpyAsync(dv, v, kb, cudaMemcpyHostToDevice, stream);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(dcq, cu_seqlens_q, cb, cudaMemcpyHostToDevice, stream);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(dck, cu_seqlens_k, cb, cudaMemcpyHostToDevice, stream);
-    if (e != cudaSuccess) {
-        cudaFreeAsync(ws, stream);
-        return cuda_fail(e, "host-to-device copy");
+    if (n > 1) {
+        ev.resize(2 * n + 3, nullptr);
+        for (auto& x : ev)
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventRecord(ev[0], stream);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev[0], 0);
     }
-    Args d{dq, dk, dv, dcq, dck, batch, num_heads, num_kv_heads, max_seqlen_q, max_seqlen_k,
-           head_dim, causal ? 1 : 0, window, dout, dlse};
-    rc = forward(d, VA_PATH_AUTO, 0, stream);
-    if (rc == VA_OK && ob) e = cudaMemcpyAsync(out, dout, ob, cudaMemcpyDeviceToHost, stream);
-    if (rc == VA_OK && e == cudaSuccess && lb)
-        e = cudaMemcpyAsync(lse, dlse, lb, cudaMemcpyDeviceToHost, stream);
+    // every host-to-device copy, chunk after chunk, on the input stream
+    if (e == cudaSuccess && cb) e = cudaMemcpyAsync(dcu, cu_h.data(), cb, cudaMemcpyHostToDevice, s_in);
+    for (int c = 0; c < n && e == cudaSuccess; ++c) {
+        const size_t r0 = cu_seqlens_q[bounds[c]], r1 = cu_seqlens_q[bounds[c + 1]];
+        const size_t k0 = cu_seqlens_k[bounds[c]], k1 = cu_seqlens_k[bounds[c + 1]];
+        if (r1 > r0)
+            e = cudaMemcpyAsync(dq + r0 * q_row, static_cast<const char*>(q) + r0 * q_row,
+                                (r1 - r0) * q_row, cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess && k1 > k0)
+            e = cudaMemcpyAsync(dk + k0 * k_row, static_cast<const char*>(k) + k0 * k_row,
+                                (k1 - k0) * k_row, cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess && k1 > k0)
+            e = cudaMemcpyAsync(dv + k0 * k_row, static_cast<const char*>(v) + k0 * k_row,
+                                (k1 - k0) * k_row, cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess && n > 1) e = cudaEventRecord(ev[1 + c], s_in);
+    }
+    // chunk by chunk: its kernels on the caller's stream, then its results
+    // back on the output stream
+    for (int c = 0; c < n && e == cudaSuccess && rc == VA_OK; ++c) {
+        const size_t r0 = cu_seqlens_q[bounds[c]], r1 = cu_seqlens_q[bounds[c + 1]];
+        const size_t k0 = cu_seqlens_k[bounds[c]];
+        if (n > 1) e = cudaStreamWaitEvent(stream, ev[1 + c], 0);
+        if (e != cudaSuccess) break;
+        Args d{dq + r0 * q_row, dk + k0 * k_row, dv + k0 * k_row, dcu + bounds[c] + c,
+               dcu + batch + n + bounds[c] + c, bounds[c + 1] - bounds[c], num_heads, num_kv_heads,
+               max_seqlen_q, max_seqlen_k, head_dim, causal ? 1 : 0, window, dout + r0 * q_row,
+               dlse + r0 * num_heads};
+        rc = forward(d, VA_PATH_AUTO, 0, stream);
+        if (rc != VA_OK) break;
+        if (n > 1) {
+            e = cudaEventRecord(ev[1 + n + c], stream);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev[1 + n + c], 0);
+        }
+        if (e == cudaSuccess && r1 > r0)
+            e = cudaMemcpyAsync(static_cast<char*>(out) + r0 * q_row, dout + r0 * q_row,
+                                (r1 - r0) * q_row, cudaMemcpyDeviceToHost, s_out);
+        if (e == cudaSuccess && r1 > r0)
+            e = cudaMemcpyAsync(reinterpret_cast<char*>(lse) + r0 * l_row,
+                                reinterpret_cast<char*>(dlse) + r0 * l_row, (r1 - r0) * l_row,
+                                cudaMemcpyDeviceToHost, s_out);
+    }
+    // the caller's stream waits for both copy streams (also after an error,
+    // so that nothing still reads the workspace when it is freed)
+    if (n > 1) {
+        cudaError_t w = (ev[2 * n + 1] && ev[2 * n + 2]) ? cudaSuccess : cudaErrorInvalidResourceHandle;
+        if (w == cudaSuccess) w = cudaEventRecord(ev[2 * n + 1], s_in);
+        if (w == cudaSuccess) w = cudaStreamWaitEvent(stream, ev[2 * n + 1], 0);
+        if (w == cudaSuccess) w = cudaEventRecord(ev[2 * n + 2], s_out);
+        if (w == cudaSuccess) w = cudaStreamWaitEvent(stream, ev[2 * n + 2], 0);
+        if (w != cudaSuccess) {
+            // could not order the copy streams before the free: drain them
+            cudaStreamSynchronize(s_in);
+            cudaStreamSynchronize(s_out);
+        }
+    }
     cudaFreeAsync(ws, stream);
     cudaError_t se = cudaStreamSynchronize(stream);
+    for (auto& x : ev)
+        if (x) cudaEventDestroy(x);
     if (rc != VA_OK) return rc;
-    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+    if (e != cudaSuccess) return cuda_fail(e, "host-buffer copies");
     if (se != cudaSuccess) return cuda_fail(se, "cudaStreamSynchronize");
     return VA_OK;
 }
