@@ -248,6 +248,23 @@ int varlen_attention_device_status(unsigned* status, int clear);
  */
 int varlen_attention_selftest_wait_timeout(int32_t* gave_up, void* stream);
 
+/*
+ * Optional check of one cu_seqlens array against the preconditions the other
+ * entry points take on trust (for tests and debugging; no other entry point
+ * calls it).  cu_seqlens has batch + 1 int32 entries, in host memory
+ * (on_device = 0) or in device memory (on_device != 0: copied to the host on
+ * `stream`, which is then synchronised).  Checks that cu_seqlens[0] == 0,
+ * that the entries never decrease, that no sequence is longer than
+ * max_seqlen and, when total >= 0, that cu_seqlens[batch] == total: the
+ * packed layout of boostr varlen_attention.rs, VarLenAttentionOps docs
+ * ("Layout contract": cumulative sequence lengths starting at 0).  Returns
+ * VA_OK, or VA_ERR_INVALID_ARG with a message naming the first offending
+ * entry (NULL pointer, batch < 0 or max_seqlen < 0 included); VA_ERR_CUDA if
+ * the copy fails.  Reads nothing past entry batch.
+ */
+int varlen_attention_validate_cu_seqlens(const int32_t* cu_seqlens, int batch, int max_seqlen,
+                                         int total, int on_device, void* stream);
+
 /* Message for the last non-VA_OK return on this host thread ("" if none). */
 const char* varlen_attention_last_error(void);
 

@@ -82,3 +82,36 @@ def test_kvcache_entry_requires_seqused_without_gpu(lib):
                                           None)
     assert rc == -1
     assert b"seqused_k is NULL" in lib.varlen_attention_last_error()
+
+
+@pytest.mark.parametrize("cu,batch,max_len,total,needle", [
+    ([0, 512, 812, 940], 3, 512, 940, None),        # the worked example's offsets
+    ([0, 512, 812, 940], 3, 512, -1, None),         # total not checked
+    ([0, 0, 7, 7], 3, 7, 7, None),                  # empty sequences
+    ([0], 0, 0, 0, None),                           # empty batch
+    ([1, 512, 812, 940], 3, 512, -1, "cu_seqlens[0] = 1"),
+    ([0, 512, 500, 940], 3, 512, -1, "decreases at entry 2"),
+    ([0, 512, 812, 940], 3, 511, -1, "sequence 0 has length 512"),
+    ([0, 512, 812, 940], 3, 512, 941, "expected the total 941"),
+])
+def test_validate_cu_seqlens_host_arrays(lib, cu, batch, max_len, total, needle):
+    import torch
+    t = torch.tensor(cu + [-5], dtype=torch.int32)   # a trailing entry the check must not read
+    rc = lib.varlen_attention_validate_cu_seqlens(t.data_ptr(), batch, max_len, total, 0, None)
+    if needle is None:
+        assert rc == 0, lib.varlen_attention_last_error().decode()
+        binding.validate_cu_seqlens(t, batch, max_len, total)
+    else:
+        assert rc == -1
+        assert needle in lib.varlen_attention_last_error().decode()
+        with pytest.raises(binding.VarlenAttentionError):
+            binding.validate_cu_seqlens(t, batch, max_len, total)
+
+
+def test_validate_cu_seqlens_rejects_bad_arguments(lib):
+    assert lib.varlen_attention_validate_cu_seqlens(None, 1, 8, -1, 0, None) == -1
+    assert b"NULL" in lib.varlen_attention_last_error()
+    import torch
+    t = torch.tensor([0, 4], dtype=torch.int32)
+    assert lib.varlen_attention_validate_cu_seqlens(t.data_ptr(), -1, 8, -1, 0, None) == -1
+    assert lib.varlen_attention_validate_cu_seqlens(t.data_ptr(), 1, -1, -1, 0, None) == -1

@@ -128,6 +128,19 @@ def test_host_buffer_entry_matches_device_entry():
     assert torch.equal(out_h, out_d.cpu()) and torch.equal(lse_h, lse_d.cpu())
 
 
+def test_validate_cu_seqlens_device_array_matches_host_array():
+    for cu, max_len, ok in (([0, 512, 812, 940], 512, True), ([0, 512, 500, 940], 512, False)):
+        host = torch.tensor(cu, dtype=torch.int32)
+        dev = host.cuda()
+        for t in (host, dev):
+            if ok:
+                binding.validate_cu_seqlens(t, 3, max_len, 940)
+            else:
+                with pytest.raises(binding.VarlenAttentionError) as e:
+                    binding.validate_cu_seqlens(t, 3, max_len, 940)
+                assert "decreases at entry 2" in str(e.value)
+
+
 def test_host_buffer_entry_pipelined_chunks_match_device_entry():
     # inputs above the pipelining threshold: the host entry splits the batch
     # into chunks of whole sequences, each copied in, computed and copied out

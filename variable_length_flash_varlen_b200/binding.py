@@ -34,6 +34,7 @@ SIGNATURES = {
     "varlen_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_schedule": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P]),
     "varlen_attention_device_status": (_I, [ctypes.POINTER(ctypes.c_uint), _I]),
+    "varlen_attention_validate_cu_seqlens": (_I, [_P, _I, _I, _I, _I, _P]),
     "varlen_attention_selftest_wait_timeout": (_I, [_P, _P]),
     "varlen_attention_last_error": (ctypes.c_char_p, []),
     "varlen_attention_version": (_I, []),
@@ -284,6 +285,20 @@ def varlen_attention_schedule(cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Te
                                          _stream_ptr(stream)))
     torch.cuda.current_stream().synchronize() if stream is None else stream.synchronize()
     return tiles[: int(n.item())]
+
+
+def validate_cu_seqlens(cu_seqlens: torch.Tensor, batch: int, max_seqlen: int, total: int = -1,
+                        stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Check a cu_seqlens array (int32, host or device) against the layout's
+    preconditions; raises VarlenAttentionError naming the first bad entry."""
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous():
+        raise ValueError("cu_seqlens must be a contiguous int32 tensor")
+    if cu_seqlens.numel() < batch + 1:
+        raise ValueError(f"cu_seqlens has {cu_seqlens.numel()} entries, batch {batch} needs {batch + 1}")
+    on_device = cu_seqlens.is_cuda
+    _check(load().varlen_attention_validate_cu_seqlens(
+        cu_seqlens.data_ptr(), batch, max_seqlen, total, int(on_device),
+        _stream_ptr(stream) if on_device else None))
 
 
 def device_status(clear: bool = True) -> int:

@@ -871,6 +871,38 @@ int varlen_attention_schedule(const int32_t* cu_seqlens_q, const int32_t* cu_seq
     return VA_OK;
 }
 
+int varlen_attention_validate_cu_seqlens(const int32_t* cu_seqlens, int batch, int max_seqlen,
+                                         int total, int on_device, void* stream_) {
+    g_last_error[0] = 0;
+    if (!cu_seqlens) return fail(VA_ERR_INVALID_ARG, "cu_seqlens is NULL");
+    if (batch < 0) return fail(VA_ERR_INVALID_ARG, "batch must be >= 0 (got %d)", batch);
+    if (max_seqlen < 0) return fail(VA_ERR_INVALID_ARG, "max_seqlen must be >= 0 (got %d)", max_seqlen);
+    std::vector<int32_t> host;
+    const int32_t* c = cu_seqlens;
+    if (on_device) {
+        host.resize(static_cast<size_t>(batch) + 1);
+        cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+        VA_CUDA(cudaMemcpyAsync(host.data(), cu_seqlens, host.size() * sizeof(int32_t),
+                                cudaMemcpyDeviceToHost, stream));
+        VA_CUDA(cudaStreamSynchronize(stream));
+        c = host.data();
+    }
+    if (c[0] != 0) return fail(VA_ERR_INVALID_ARG, "cu_seqlens[0] = %d, must be 0", c[0]);
+    for (int b = 0; b < batch; ++b) {
+        const long long len = static_cast<long long>(c[b + 1]) - c[b];
+        if (len < 0)
+            return fail(VA_ERR_INVALID_ARG, "cu_seqlens decreases at entry %d (%d -> %d)", b + 1,
+                        c[b], c[b + 1]);
+        if (len > max_seqlen)
+            return fail(VA_ERR_INVALID_ARG, "sequence %d has length %lld > max_seqlen %d", b, len,
+                        max_seqlen);
+    }
+    if (total >= 0 && c[batch] != total)
+        return fail(VA_ERR_INVALID_ARG, "cu_seqlens[%d] = %d, expected the total %d", batch,
+                    c[batch], total);
+    return VA_OK;
+}
+
 int varlen_attention_device_status(unsigned* status, int clear) {
     g_last_error[0] = 0;
     if (!status) return fail(VA_ERR_INVALID_ARG, "status is NULL");
