@@ -1,16 +1,20 @@
 """Benchmark of the packed variable-length attention forward on B200.
 
 Prints ONE JSON line (rank 0).  Metric: prefill TFLOP/s of the varlen forward
-(algorithmic FLOPs = 4 * visible (q, k) pairs * D * H) on the 16-sequence
-non-causal MHA workload (q = k lengths uniform-int in [64, 2048], H = H_kv =
-16, D = 128), with the decode-shape HBM GB/s (128 sequences of one query,
-k lengths uniform-int in [1024, 32768], H = 32, H_kv = 8, D = 128) reported
-beside it under "decode", the chunked-prefill workload under
-"chunked_prefill", the same headline workload in FP8 (E4M3 inputs and
-output with per-tensor scales, varlen_attention_fwd_fp8) under "fp8" and its
-backward pass (varlen_attention_bwd) under "backward".  A step
-is one call of the C ABI on one batch: schedule build + prefill kernel
-(decode: split + combine kernels).
+(algorithmic FLOPs = 4 * visible (q, k) pairs * D * H) with its fraction of
+the bf16 tensor peak, headlined on the largest configuration, the sliding
+window (4 sequences of 32768 tokens, window 4096, causal, H=32, H_kv=8,
+D=128, 8.25 TFLOP per call).  Beside it: every other prefill configuration
+(the worked example, the 16-sequence non-causal MHA workload, the GQA causal
+workload) under "prefill_configs", the decode-shape HBM GB/s (128 sequences
+of one query, k lengths uniform-int in [1024, 32768], H=32, H_kv=8, D=128)
+under "decode", the chunked-prefill workload under "chunked_prefill", the MHA
+workload in FP8 (E4M3 inputs and output with per-tensor scales,
+varlen_attention_fwd_fp8) under "fp8", the backward pass (varlen_attention_bwd)
+on the MHA and GQA workloads under "backward", and the headline end to end
+through the host-buffer entry point under "e2e".  A step is one call of the C
+ABI on one batch: schedule build + prefill kernel (decode: split + combine
+kernels).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload NAME]
@@ -38,6 +42,10 @@ sys.path.insert(0, ROOT)
 from variable_length_flash_varlen_b200 import accounting, binding, workloads  # noqa: E402
 
 METRIC = "varlen FA fwd TFLOP/s + % BF16 TC peak; decode-shape HBM GB/s + % peak"
+# every prefill configuration of the metric, each timed in its own loop; the
+# headline (--workload) is the largest one that fits one GPU
+PREFILL_CONFIGS = ("worked_example", "mha_noncausal", "gqa_causal", "sliding_window")
+BACKWARD_CONFIGS = ("mha_noncausal", "gqa_causal")
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -53,13 +61,12 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-# Sources each kernel is compiled from (the launch code in varlen_attn.cu
-# included), so a recorded traffic figure goes stale only when its own kernel
-# changes.
+# Device sources each kernel is compiled from (its block size, shared memory
+# and launch shape are constants of these headers; the grid is one CTA per SM),
+# so a recorded traffic figure goes stale only when its own kernel changes.
 KERNEL_SOURCES = {
-    "prefill_fwd_kernel": ("prefill_sm100.cuh", "f32x2.cuh", "schedule.cuh", "ptx.cuh", "status.cuh",
-                           "varlen_attn.cu"),
-    "decode_stream_kernel": ("decode.cuh", "schedule.cuh", "ptx.cuh", "status.cuh", "varlen_attn.cu"),
+    "prefill_fwd_kernel": ("prefill_sm100.cuh", "f32x2.cuh", "schedule.cuh", "ptx.cuh", "status.cuh"),
+    "decode_stream_kernel": ("decode.cuh", "schedule.cuh", "ptx.cuh", "status.cuh"),
 }
 
 
@@ -296,6 +303,12 @@ def run_profile_target(args, local):
     binding.load()
     name = "decode" if args.only == "decode" else args.workload
     wl = workloads.named(name, scale=args.scale)
+    if args.first_seqs > 0:
+        # the first N sequences alone (a smaller capture whose work, and traffic,
+        # is the full workload's share of those sequences)
+        n = args.first_seqs
+        wl = workloads.custom(wl.lengths_q[:n], wl.lengths_k[:n], wl.H, wl.H_kv, wl.D, wl.causal,
+                              wl.window, wl.seed, name=wl.name)
     if args.only == "fp8":
         q8, k8, v8, sc = workloads.make_qkv_fp8(wl)
         d8 = [t.to(dev) for t in (q8, k8, v8)]
@@ -338,119 +351,141 @@ def run_profile_target(args, local):
         raise SystemExit("device status word raised")
 
 
+def _inputs_on(wl, dev):
+    q, k, v = workloads.make_qkv(wl)
+    cq = torch.tensor(wl.cu_q, dtype=torch.int32, device=dev)
+    ck = torch.tensor(wl.cu_k, dtype=torch.int32, device=dev)
+    return (q, k, v), (q.to(dev), k.to(dev), v.to(dev), cq, ck)
+
+
+def _fwd_call(wl, d, out, lse):
+    dq, dk, dv, cq, ck = d
+    return lambda: binding.varlen_attention_fwd(dq, dk, dv, cq, ck, wl.batch, wl.H, wl.H_kv,
+                                                wl.max_seqlen_q, wl.max_seqlen_k, wl.D, wl.causal,
+                                                wl.window, out=out, lse=lse)
+
+
+def _tensor_roofline(achieved, peak, peak_kind, **extra):
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "peak_kind": peak_kind, **extra}
+
+
 def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     peaks, peak_kind = load_peaks()
+    peak = peaks["bf16_tflops"]
+    pk = f"{peak_kind} bf16 burst"
     binding.load()
-
-    # ---- prefill workload (the headline)
-    wl = workloads.named(args.workload, seed=workloads.WORKLOAD_SEEDS[args.workload] + rank)
-    q, k, v = workloads.make_qkv(wl)
-    dq, dk, dv = q.to(dev), k.to(dev), v.to(dev)
-    cq = torch.tensor(wl.cu_q, dtype=torch.int32, device=dev)
-    ck = torch.tensor(wl.cu_k, dtype=torch.int32, device=dev)
-    out = torch.empty_like(dq)
-    lse = torch.empty(wl.total_q, wl.H, dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    flops = accounting.attention_flops(wl)
-
-    def step():
-        binding.varlen_attention_fwd(dq, dk, dv, cq, ck, wl.batch, wl.H, wl.H_kv, wl.max_seqlen_q,
-                                     wl.max_seqlen_k, wl.D, wl.causal, wl.window, out=out, lse=lse)
+    seed = lambda name: workloads.WORKLOAD_SEEDS[name] + rank  # noqa: E731
 
     visible = os.environ.get("CUDA_VISIBLE_DEVICES")
     smi_index = int(visible.split(",")[local]) if visible and visible.split(",")[local].isdigit() else local
-    # clocks are sampled across all timed loops (prefill, decode, chunked prefill, end to end)
+    # clocks are sampled across all timed loops
     clk = ClockSampler(smi_index if not args.no_clock_sampler else None).__enter__()
-    step_ms, outer_ms = time_device_steps(step, args.steps, args.warmup, flush, world, stream)
-    t_local = sum(step_ms) / 1e3
-    t_max = max_over_ranks(t_local, world)
-    total_flops = sum_over_ranks(flops * args.steps, world)
-    value = total_flops / t_max / 1e12
-    per_launch_s = t_local / args.steps
-    achieved = flops / per_launch_s / 1e12
-    peak = peaks["bf16_tflops"]
+
+    def timed(fn):
+        ms, _ = time_device_steps(fn, args.steps, args.warmup, flush, world, stream)
+        local_s = sum(ms) / 1e3
+        return ms, local_s, max_over_ranks(local_s, world)
+
+    def prefill_leg(name):
+        wl = workloads.named(name, seed=seed(name))
+        host, d = _inputs_on(wl, dev)
+        out = torch.empty_like(d[0])
+        lse = torch.empty(wl.total_q, wl.H, dtype=torch.float32, device=dev)
+        flops = accounting.attention_flops(wl)
+        ms, local_s, max_s = timed(_fwd_call(wl, d, out, lse))
+        value = sum_over_ranks(flops * args.steps, world) / max_s / 1e12
+        achieved = flops / (local_s / args.steps) / 1e12
+        return wl, host, d, (out, lse), {
+            "workload": name, **wl.describe(), "value": value, "unit": "TFLOP/s",
+            "ms_per_step": max_s / args.steps * 1e3, "flops_per_step_per_gpu": flops,
+            "roofline": _tensor_roofline(achieved, peak, pk,
+                                         kernel=f"prefill_fwd_kernel<{wl.D}> (+ schedule build, same call)",
+                                         traffic=recorded_traffic("prefill_fwd_kernel", name)),
+            "gpu_launches": 2 * args.steps}, ms
+
+    # ---- the headline: prefill TFLOP/s on the largest configuration (sliding window)
+    wl, host, d, (out, lse), head, step_ms = prefill_leg(args.workload)
+    q, k, v = host
+
+    # ---- the other prefill configurations, each its own timed loop
+    prefill_configs = {}
+    for name in PREFILL_CONFIGS:
+        if name != args.workload:
+            r = prefill_leg(name)
+            prefill_configs[name] = r[4]
+            del r
 
     # ---- decode workload (the HBM half of the metric)
-    dwl = workloads.named("decode", seed=workloads.WORKLOAD_SEEDS["decode"] + rank)
-    qd, kd, vd = workloads.make_qkv(dwl)
-    dqd, dkd, dvd = qd.to(dev), kd.to(dev), vd.to(dev)
-    cqd = torch.tensor(dwl.cu_q, dtype=torch.int32, device=dev)
-    ckd = torch.tensor(dwl.cu_k, dtype=torch.int32, device=dev)
-    outd = torch.empty_like(dqd)
+    dwl = workloads.named("decode", seed=seed("decode"))
+    _, dd = _inputs_on(dwl, dev)
+    outd = torch.empty_like(dd[0])
     lsed = torch.empty(dwl.total_q, dwl.H, dtype=torch.float32, device=dev)
-
-    def dstep():
-        binding.varlen_attention_fwd(dqd, dkd, dvd, cqd, ckd, dwl.batch, dwl.H, dwl.H_kv,
-                                     dwl.max_seqlen_q, dwl.max_seqlen_k, dwl.D, dwl.causal,
-                                     dwl.window, out=outd, lse=lsed)
-
-    d_ms, _ = time_device_steps(dstep, args.steps, args.warmup, flush, world, stream)
-    d_local = sum(d_ms) / 1e3
-    d_max = max_over_ranks(d_local, world)
+    _, d_local, d_max = timed(_fwd_call(dwl, dd, outd, lsed))
     dbytes = accounting.decode_bytes(dwl)
     d_value = sum_over_ranks(dbytes * args.steps, world) / d_max / 1e9
-    del dqd, dkd, dvd, outd, lsed
+    del dd, outd, lsed
 
     # ---- chunked prefill: new query chunks after cached prefixes (L_q < L_k, causal)
-    cwl = workloads.named("chunked_prefill", seed=workloads.WORKLOAD_SEEDS["chunked_prefill"] + rank)
-    qc, kc, vc = workloads.make_qkv(cwl)
-    dqc, dkc, dvc = qc.to(dev), kc.to(dev), vc.to(dev)
-    cqc = torch.tensor(cwl.cu_q, dtype=torch.int32, device=dev)
-    ckc = torch.tensor(cwl.cu_k, dtype=torch.int32, device=dev)
-    outc = torch.empty_like(dqc)
-    lsec = torch.empty(cwl.total_q, cwl.H, dtype=torch.float32, device=dev)
+    chunked = prefill_leg("chunked_prefill")[4]
 
-    def cstep():
-        binding.varlen_attention_fwd(dqc, dkc, dvc, cqc, ckc, cwl.batch, cwl.H, cwl.H_kv,
-                                     cwl.max_seqlen_q, cwl.max_seqlen_k, cwl.D, cwl.causal,
-                                     cwl.window, out=outc, lse=lsec)
-
-    c_ms, _ = time_device_steps(cstep, args.steps, args.warmup, flush, world, stream)
-    c_max = max_over_ranks(sum(c_ms) / 1e3, world)
-    cflops = accounting.attention_flops(cwl)
-    c_value = sum_over_ranks(cflops * args.steps, world) / c_max / 1e12
-    del dqc, dkc, dvc, outc, lsec, qc, kc, vc
-
-    # ---- FP8 (E4M3) forward on the headline workload (flash_attention_fwd_fp8 semantics)
-    fq, fk, fv, fsc = workloads.make_qkv_fp8(wl)
+    # ---- FP8 (E4M3) forward on the MHA workload (flash_attention_fwd_fp8 semantics)
+    fwl = workloads.named("mha_noncausal", seed=seed("mha_noncausal"))
+    fq, fk, fv, fsc = workloads.make_qkv_fp8(fwl)
     dfq, dfk, dfv = fq.to(dev), fk.to(dev), fv.to(dev)
+    fcq = torch.tensor(fwl.cu_q, dtype=torch.int32, device=dev)
+    fck = torch.tensor(fwl.cu_k, dtype=torch.int32, device=dev)
     fout = torch.empty_like(dfq)
-    flse = torch.empty(wl.total_q, wl.H, dtype=torch.float32, device=dev)
+    flse = torch.empty(fwl.total_q, fwl.H, dtype=torch.float32, device=dev)
 
     def fstep():
-        binding.varlen_attention_fwd_fp8(dfq, dfk, dfv, cq, ck, wl.batch, wl.H, wl.H_kv,
-                                         wl.max_seqlen_q, wl.max_seqlen_k, wl.D, wl.causal,
-                                         wl.window, fsc["q_scale"], fsc["k_scale"], fsc["v_scale"],
+        binding.varlen_attention_fwd_fp8(dfq, dfk, dfv, fcq, fck, fwl.batch, fwl.H, fwl.H_kv,
+                                         fwl.max_seqlen_q, fwl.max_seqlen_k, fwl.D, fwl.causal,
+                                         fwl.window, fsc["q_scale"], fsc["k_scale"], fsc["v_scale"],
                                          fsc["o_scale"], out=fout, lse=flse)
 
-    f_ms, _ = time_device_steps(fstep, args.steps, args.warmup, flush, world, stream)
-    f_max = max_over_ranks(sum(f_ms) / 1e3, world)
-    f_value = total_flops / f_max / 1e12
+    _, _, f_max = timed(fstep)
+    fflops = accounting.attention_flops(fwl)
+    f_value = sum_over_ranks(fflops * args.steps, world) / f_max / 1e12
     # E4M3 dense tensor peak: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
     fp8_peak = peak * 2.0
     del dfq, dfk, dfv, fout, flse, fq, fk, fv
 
-    # ---- backward pass on the headline workload (dq, dk, dv from the forward's out and lse)
-    gen = torch.Generator().manual_seed(workloads.WORKLOAD_SEEDS[args.workload] + 7 + rank)
-    ddo = torch.randn(wl.total_q, wl.H, wl.D, generator=gen).to(torch.bfloat16).to(dev)
-    binding.varlen_attention_fwd(dq, dk, dv, cq, ck, wl.batch, wl.H, wl.H_kv, wl.max_seqlen_q,
-                                 wl.max_seqlen_k, wl.D, wl.causal, wl.window, out=out, lse=lse)
-    gq, gk, gv = torch.empty_like(dq), torch.empty_like(dk), torch.empty_like(dv)
+    # ---- backward pass (dq, dk, dv from the forward's out and lse) on two workloads
+    backward = {}
+    for name in BACKWARD_CONFIGS:
+        bwl = workloads.named(name, seed=seed(name))
+        _, bd = _inputs_on(bwl, dev)
+        bq, bk, bv, bcq, bck = bd
+        gen = torch.Generator().manual_seed(workloads.WORKLOAD_SEEDS[name] + 7 + rank)
+        ddo = torch.randn(bwl.total_q, bwl.H, bwl.D, generator=gen).to(torch.bfloat16).to(dev)
+        bout = torch.empty_like(bq)
+        blse = torch.empty(bwl.total_q, bwl.H, dtype=torch.float32, device=dev)
+        _fwd_call(bwl, bd, bout, blse)()
+        gq, gk, gv = torch.empty_like(bq), torch.empty_like(bk), torch.empty_like(bv)
 
-    def bstep():
-        binding.varlen_attention_bwd(ddo, dq, dk, dv, out, lse, cq, ck, wl.batch, wl.H, wl.H_kv,
-                                     wl.max_seqlen_q, wl.max_seqlen_k, wl.D, wl.causal, wl.window,
-                                     dq=gq, dk=gk, dv=gv)
+        def bstep():
+            binding.varlen_attention_bwd(ddo, bq, bk, bv, bout, blse, bcq, bck, bwl.batch, bwl.H,
+                                         bwl.H_kv, bwl.max_seqlen_q, bwl.max_seqlen_k, bwl.D,
+                                         bwl.causal, bwl.window, dq=gq, dk=gk, dv=gv)
 
-    b_ms, _ = time_device_steps(bstep, args.steps, args.warmup, flush, world, stream)
-    b_max = max_over_ranks(sum(b_ms) / 1e3, world)
-    bflops = accounting.backward_flops(wl)
-    b_value = sum_over_ranks(bflops * args.steps, world) / b_max / 1e12
-    del ddo, gq, gk, gv
+        _, _, b_max = timed(bstep)
+        bflops = accounting.backward_flops(bwl)
+        b_value = sum_over_ranks(bflops * args.steps, world) / b_max / 1e12
+        backward[name] = {
+            "workload": name, "entry": "varlen_attention_bwd", "value": b_value, "unit": "TFLOP/s",
+            "ms_per_step": b_max / args.steps * 1e3, "flops_per_step_per_gpu": bflops,
+            "roofline": _tensor_roofline(b_value / world, peak, pk,
+                                         kernel="bwd_dq_kernel + bwd_dkdv_kernel (same call)"),
+            "gpu_launches": 2 * args.steps}
+        del bd, bq, bk, bv, ddo, bout, blse, gq, gk, gv
 
-    # ---- end to end through the host-buffer entry point (pinned memory)
+    # ---- end to end on the headline workload through the host-buffer entry point
+    # (pinned memory; copies in and out inside the timed region)
+    del d
     qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
     cqh = torch.tensor(wl.cu_q, dtype=torch.int32)
     ckh = torch.tensor(wl.cu_k, dtype=torch.int32)
@@ -462,10 +497,10 @@ def run_ours(args, world, rank, local):
                                           wl.max_seqlen_q, wl.max_seqlen_k, wl.D, wl.causal,
                                           wl.window, outh, lseh)
 
-    e_ms, _ = time_device_steps(estep, args.steps, args.warmup, flush, world, stream)
+    _, _, e_max = timed(estep)
     clk.__exit__(None, None, None)
-    e_max = max_over_ranks(sum(e_ms) / 1e3, world)
-    e_value = total_flops / e_max / 1e12
+    flops = head["flops_per_step_per_gpu"]
+    e_value = sum_over_ranks(flops * args.steps, world) / e_max / 1e12
     h2d = (q.numel() + k.numel() + v.numel()) * 2 + (len(wl.cu_q) + len(wl.cu_k)) * 4
     d2h = out.numel() * 2 + lse.numel() * 4
 
@@ -481,18 +516,19 @@ def run_ours(args, world, rank, local):
 
     clocks = clk.summary()
     d_frac = d_value / (peaks["hbm_gbs"] * world)
+    config = {k2: v2 for k2, v2 in head.items()
+              if k2 not in ("value", "unit", "ms_per_step", "roofline", "gpu_launches")}
+    config.update({"parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2, and a 256 MiB buffer written before every step, "
+                         "outside the step events"})
     return {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_max / args.steps * 1e3,
+        "metric": METRIC, "value": head["value"], "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": args.workload, **wl.describe(), "parallelism": f"dp{world}",
-                   "l2": "256 MiB buffer written before every step, outside the step events",
-                   "flops_per_step_per_gpu": flops},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "peak_kind": f"{peak_kind} bf16 burst",
-                     "kernel": "prefill_fwd_kernel<128> (+ schedule build, same call)",
-                     "traffic": recorded_traffic("prefill_fwd_kernel", args.workload)},
+        "config": config,
+        "roofline": head["roofline"],
+        "prefill_configs": prefill_configs,
         "decode": {"workload": "decode", **dwl.describe(), "value": d_value, "unit": "GB/s",
                    "ms_per_step": d_max / args.steps * 1e3, "bytes_per_step": dbytes,
                    "roofline": {"bound": "hbm", "achieved": d_value / world,
@@ -501,34 +537,22 @@ def run_ours(args, world, rank, local):
                                 "kernel": "decode_stream_kernel<128> (+ combine and counter reset, same call)",
                                 "traffic": recorded_traffic("decode_stream_kernel", "decode")},
                    "gpu_launches": 2 * args.steps},
-        "chunked_prefill": {**cwl.describe(), "value": c_value, "unit": "TFLOP/s",
-                            "ms_per_step": c_max / args.steps * 1e3, "flops_per_step_per_gpu": cflops,
-                            "roofline": {"bound": "tensor", "achieved": c_value / world, "peak": peak,
-                                         "unit": "TFLOP/s", "frac": c_value / world / peak,
-                                         "peak_kind": f"{peak_kind} bf16 burst"},
-                            "gpu_launches": 2 * args.steps},
-        "fp8": {"workload": args.workload, "entry": "varlen_attention_fwd_fp8", "dtype": "e4m3",
+        "chunked_prefill": chunked,
+        "fp8": {"workload": "mha_noncausal", "entry": "varlen_attention_fwd_fp8", "dtype": "e4m3",
                 "scales": fsc, "value": f_value, "unit": "TFLOP/s",
-                "ms_per_step": f_max / args.steps * 1e3,
+                "ms_per_step": f_max / args.steps * 1e3, "flops_per_step_per_gpu": fflops,
                 "roofline": {"bound": "tensor", "achieved": f_value / world, "peak": fp8_peak,
                              "unit": "TFLOP/s", "frac": f_value / world / fp8_peak,
                              "peak_kind": f"{peak_kind} bf16 burst x 2 (nominal e4m3 / bf16 ratio)",
                              "kernel": "prefill_fwd_kernel<128, E4M3> (+ schedule build, same call)"},
                 "gpu_launches": 2 * args.steps},
-        "backward": {"workload": args.workload, "entry": "varlen_attention_bwd", "value": b_value,
-                     "unit": "TFLOP/s", "ms_per_step": b_max / args.steps * 1e3,
-                     "flops_per_step_per_gpu": bflops,
-                     "roofline": {"bound": "tensor", "achieved": b_value / world, "peak": peak,
-                                  "unit": "TFLOP/s", "frac": b_value / world / peak,
-                                  "peak_kind": f"{peak_kind} bf16 burst",
-                                  "kernel": "bwd_delta + bwd_dkdv + bwd_dq (same call)"},
-                     "gpu_launches": 3 * args.steps},
+        "backward": backward,
         "e2e": {"value": e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h, "entry": "varlen_attention_fwd_host",
+                "workload": args.workload},
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
-        "outer_ms_with_flush": outer_ms,
         "step_ms": [round(x, 4) for x in step_ms],
     }
 
@@ -539,12 +563,14 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="mha_noncausal", choices=list(workloads.WORKLOAD_SEEDS))
+    ap.add_argument("--workload", default="sliding_window", choices=list(workloads.WORKLOAD_SEEDS))
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--no-clock-sampler", action="store_true")
     ap.add_argument("--scale", type=float, default=1.0,
                     help="shrink every sequence length (profiling captures of a small case)")
+    ap.add_argument("--first-seqs", type=int, default=0,
+                    help="profiling: keep only the first N sequences of the workload")
     ap.add_argument("--only", choices=["all", "prefill", "fp8", "bwd", "decode"], default="all",
                     help="profiling: run only one half of the step (no JSON line)")
     args = ap.parse_args()

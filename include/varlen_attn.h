@@ -32,8 +32,9 @@
  * NULL = the legacy default stream) and never synchronises; cu_seqlens stay
  * on the device.  Launch errors are returned; device-side conditions (a
  * bounded barrier wait that gave up, more query tiles than max_seqlen_q
- * allows for) set bits in a device status word read by
- * varlen_attention_device_status().
+ * allows for) set bits in a device status word, which
+ * varlen_attention_sync_status() reads in the order of one stream (and
+ * varlen_attention_device_status() after a device-wide synchronisation).
  *
  * Preconditions not checked on the device: cu arrays are non-decreasing with
  * cu[0] = 0; max_seqlen_q / max_seqlen_k are >= every L_q / L_k (they size
@@ -57,6 +58,7 @@ extern "C" {
 #define VA_ERR_INVALID_ARG (-1) /* null pointer, negative size, H % H_kv != 0, misalignment */
 #define VA_ERR_UNSUPPORTED (-2) /* head_dim other than 64 or 128, sizes beyond int32 indexing */
 #define VA_ERR_CUDA (-3)        /* a CUDA runtime / driver call or a launch failed */
+#define VA_ERR_DEVICE_TIMEOUT (-4) /* a bounded wait inside a kernel gave up (status queries) */
 
 /* Device status bits (varlen_attention_device_status). */
 #define VA_STATUS_WAIT_TIMEOUT 1u       /* a bounded wait inside a kernel gave up */
@@ -182,7 +184,12 @@ int varlen_attention_fwd_ex(const void* q, const void* k, const void* v,
  * run on `stream` while the next chunk is copied in and the previous one
  * copied out on two library-owned copy streams (created on the first such
  * call per device); the results are bit-identical to one launch over the
- * whole batch.
+ * whole batch.  Because both cu_seqlens arrays are in host memory here, the
+ * call checks them before any device work (the checks of
+ * varlen_attention_validate_cu_seqlens: cu[0] == 0, never decreasing, no
+ * sequence longer than max_seqlen_q / max_seqlen_k, cu_seqlens_q[batch]
+ * and cu_seqlens_k[batch] are the packed totals the copies read) and
+ * returns VA_ERR_INVALID_ARG naming the first bad entry.
  */
 int varlen_attention_fwd_host(const void* q, const void* k, const void* v,
                               const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
@@ -237,6 +244,25 @@ int varlen_attention_schedule(const int32_t* cu_seqlens_q, const int32_t* cu_seq
 int varlen_attention_device_status(unsigned* status, int clear);
 
 /*
+ * Stream-scoped status query: the device status word as seen after the work
+ * already enqueued on `stream` (a cudaStream_t of the current device, NULL =
+ * the legacy default stream).  Enqueues a copy of the word on `stream`,
+ * synchronises that stream only (other streams keep running), stores the
+ * word in *status (VA_STATUS_* bits) and, if clear != 0, resets it with a
+ * write enqueued on `stream` after the copy.  The word is one per device,
+ * shared by all streams: a bit raised by work on another stream shows up
+ * here too once that work has finished.
+ * Returns VA_ERR_DEVICE_TIMEOUT when VA_STATUS_WAIT_TIMEOUT is set (a
+ * kernel's bounded wait gave up: its results are incomplete),
+ * VA_ERR_INVALID_ARG when only VA_STATUS_SCHEDULE_OVERFLOW is set (a query
+ * length exceeded max_seqlen_q), VA_OK when the word is 0; VA_ERR_CUDA if a
+ * copy or the synchronisation fails, VA_ERR_INVALID_ARG for a NULL status.
+ * It blocks the calling host thread until `stream` drains, so it must not be
+ * called while `stream` is being captured into a CUDA graph.
+ */
+int varlen_attention_sync_status(void* stream, unsigned* status, int clear);
+
+/*
  * Self-test of the failure path (for tests; no fault or hang is involved).
  * Launches on `stream` a one-thread kernel that waits, through the same
  * bounded barrier wait every kernel of the library uses, on a barrier phase
@@ -250,10 +276,16 @@ int varlen_attention_selftest_wait_timeout(int32_t* gave_up, void* stream);
 
 /*
  * Optional check of one cu_seqlens array against the preconditions the other
- * entry points take on trust (for tests and debugging; no other entry point
- * calls it).  cu_seqlens has batch + 1 int32 entries, in host memory
- * (on_device = 0) or in device memory (on_device != 0: copied to the host on
- * `stream`, which is then synchronised).  Checks that cu_seqlens[0] == 0,
+ * entry points take on trust (for tests and debugging; of the other entry
+ * points only varlen_attention_fwd_host, whose arrays are already in host
+ * memory, applies the same check).  cu_seqlens has batch + 1 int32 entries,
+ * in host memory (on_device = 0) or in device memory (on_device != 0: copied
+ * to the host on `stream`, and the calling thread then blocks until `stream`
+ * drains, so a device-array check must not be made while `stream` is being
+ * captured into a CUDA graph).  For the cu_seqlens_k of
+ * varlen_attention_fwd_kvcache pass the largest slot size (the capacity
+ * stride bound) as max_seqlen, not the largest key count in use: there the
+ * steps of cu_seqlens_k are slot sizes.  Checks that cu_seqlens[0] == 0,
  * that the entries never decrease, that no sequence is longer than
  * max_seqlen and, when total >= 0, that cu_seqlens[batch] == total: the
  * packed layout of boostr varlen_attention.rs, VarLenAttentionOps docs

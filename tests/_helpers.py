@@ -5,8 +5,18 @@ import torch
 
 from variable_length_flash_varlen_b200 import binding, workloads
 
-O_TOL = 1e-2    # max |O_gpu - O_oracle| beyond the bf16 rounding of the output itself
+import os
+
+O_TOL = 1e-2    # |O_gpu - O_oracle| wherever a bf16 result can come that close
 LSE_TOL = 1e-3  # max |LSE_gpu - LSE_oracle|
+# Where |O_oracle| >= 4 the nearest bf16 number can lie up to 2^-6 = 0.0156
+# from the exact value (half the bf16 spacing there), so no bf16 output meets
+# 1e-2; there the bar is that half spacing plus this much arithmetic error.
+HALF_ULP_SLACK = 1e-3
+
+# One record per comparison, printed by the terminal summary in conftest.py:
+# (test id, elements, max |dO|, worst |dO| / bar, max |dLSE|, max |O_oracle|)
+MARGINS = []
 
 
 def bf16_half_ulp(x):
@@ -39,6 +49,18 @@ def oracle_all(oracle_lib, wl, q, k, v):
                                      wl.causal, wl.window)
 
 
+def o_bar(out_ref):
+    """Per-element bar on |O_gpu - O_oracle|: 1e-2, or where that is below
+    what any bf16 number can reach (half a bf16 step at |O_oracle| >= 4), that
+    half step plus HALF_ULP_SLACK."""
+    return np.maximum(O_TOL, bf16_half_ulp(out_ref) + HALF_ULP_SLACK)
+
+
+def record_margin(n, d_o, ratio, d_l, o_max):
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    MARGINS.append((test, int(n), float(d_o), float(ratio), float(d_l), float(o_max)))
+
+
 def compare(out_gpu, lse_gpu, out_ref, lse_ref, rows=None):
     """Element-wise comparison; returns (max |dO|, max |dLSE|)."""
     o = out_gpu.float().cpu().double().numpy()
@@ -52,10 +74,15 @@ def compare(out_gpu, lse_gpu, out_ref, lse_ref, rows=None):
     assert np.array_equal(np.isneginf(l), neg_ref), "-inf logsumexp rows differ"
     err = np.abs(o - out_ref)
     d_o = float(np.max(err)) if o.size else 0.0
-    excess = float(np.max(err - bf16_half_ulp(out_ref))) if o.size else 0.0
+    ratio = float(np.max(err / o_bar(out_ref))) if o.size else 0.0
     fin = ~neg_ref
     d_l = float(np.max(np.abs(l[fin] - lse_ref[fin]))) if fin.any() else 0.0
-    assert excess <= O_TOL, f"max |dO| = {d_o}, beyond bf16 half-ulp {excess}"
+    record_margin(o.size, d_o, ratio, d_l, float(np.max(np.abs(out_ref))) if o.size else 0.0)
+    if ratio > 1.0:
+        w = np.unravel_index(int(np.argmax(err / o_bar(out_ref))), err.shape)
+        raise AssertionError(f"|dO| beyond its bar: worst {float(err[w]):.5f} at {w} where the oracle "
+                             f"gives {float(out_ref[w]):.5f} (bar {float(o_bar(out_ref)[w]):.5f}); "
+                             f"max |dO| {d_o:.5f}")
     assert d_l <= LSE_TOL, f"max |dLSE| = {d_l}"
     return d_o, d_l
 

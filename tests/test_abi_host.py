@@ -115,3 +115,27 @@ def test_validate_cu_seqlens_rejects_bad_arguments(lib):
     t = torch.tensor([0, 4], dtype=torch.int32)
     assert lib.varlen_attention_validate_cu_seqlens(t.data_ptr(), -1, 8, -1, 0, None) == -1
     assert lib.varlen_attention_validate_cu_seqlens(t.data_ptr(), 1, -1, -1, 0, None) == -1
+
+
+@pytest.mark.parametrize("cq,ck,needle", [
+    ([0, 512, 500, 940], [0, 512, 812, 940], "cu_seqlens_q decreases at entry 2"),
+    ([0, 512, 812, 940], [3, 512, 812, 940], "cu_seqlens_k[0] = 3, must be 0"),
+    ([0, 600, 812, 940], [0, 512, 812, 940], "sequence 0 has length 600 > max_seqlen 512"),
+    ([0, 512, 812, 940], [0, 512, 812, 700], "cu_seqlens_k decreases at entry 3"),
+])
+def test_host_entry_rejects_bad_host_cu_seqlens_before_device_work(lib, cq, ck, needle):
+    # the host-buffer entry sizes its copies and chunks from these host arrays:
+    # a bad one is refused before any CUDA call (this runs without a GPU; the
+    # tensor pointers are never dereferenced)
+    import torch
+    tq = torch.tensor(cq, dtype=torch.int32)
+    tk = torch.tensor(ck, dtype=torch.int32)
+    rc = lib.varlen_attention_fwd_host(16, 16, 16, tq.data_ptr(), tk.data_ptr(), 3, 4, 2, 512, 512,
+                                       64, 1, 0, 16, 16, None)
+    assert rc == -1
+    assert needle in lib.varlen_attention_last_error().decode()
+
+
+def test_sync_status_rejects_null_pointer(lib):
+    assert lib.varlen_attention_sync_status(None, None, 0) == -1
+    assert b"status is NULL" in lib.varlen_attention_last_error()

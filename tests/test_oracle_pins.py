@@ -283,19 +283,31 @@ def test_schedule_key_ranges_match_band_mask(Lq, Lk, causal, W):
     cu_q, cu_k = workloads.cu_seqlens(Lq), workloads.cu_seqlens(Lk)
     items = sch.schedule(cu_q, cu_k, causal, W)
     BM, BN = sch.BLOCK_M, sch.BLOCK_N
-    expect = []
+    expect, few = [], set()
     for b in range(len(Lq)):
         _, keep = _band_mask(Lq[b], Lk[b], causal, W)
         for qt in range((Lq[b] + BM - 1) // BM):
-            cols = torch.nonzero(keep[qt * BM:(qt + 1) * BM].any(dim=0)).flatten()
+            rows = keep[qt * BM:(qt + 1) * BM]
+            cols = torch.nonzero(rows.any(dim=0)).flatten()
             rng = (int(cols.min()) // BN, int(cols.max()) // BN + 1) if len(cols) else (0, 0)
             expect.append((b, qt) + rng)
+            # a tile with a row that sees 1..256 keys belongs to the second part
+            counts = rows.sum(dim=1)
+            if bool(((counts >= 1) & (counts <= sch.RESIDUAL_MAX_KEYS)).any()):
+                few.add((b, qt))
     assert sorted(items) == sorted(expect)
-    costs = [it[3] - it[2] for it in items]
-    assert costs == sorted(costs, reverse=True)
-    for a, b in zip(items, items[1:]):
-        if a[3] - a[2] == b[3] - b[2]:
-            assert (a[0], a[1]) < (b[0], b[1])
+    flags = [(it[0], it[1]) in few for it in items]
+    assert flags == sorted(flags), "tiles with a few-key row must come last"
+    for part in (False, True):
+        sub = [it for it, f in zip(items, flags) if f == part]
+        costs = [it[3] - it[2] for it in sub]
+        assert costs == sorted(costs, reverse=True)
+        for a, b in zip(sub, sub[1:]):
+            if a[3] - a[2] == b[3] - b[2]:
+                assert (a[0], a[1]) < (b[0], b[1])
+    # without the split, one part ordered the same way
+    assert sch.schedule(cu_q, cu_k, causal, W, split_few_keys=False) == sorted(
+        items, key=lambda it: (-(it[3] - it[2]), it[0], it[1]))
 
 
 # --- key-value cache with a capacity stride ------------------------------------

@@ -1,8 +1,10 @@
 """GPU parity: the CUDA path through the C ABI against the fp64 oracle.
 
-Bar (element by element): max |O_gpu - O_oracle| <= 1e-2, max |LSE_gpu -
-LSE_oracle| <= 1e-3, -inf logsumexp exactly where the oracle has one, no NaN;
-the tile work list bit-exact against the CPU statement in oracle/schedule.py.
+Bar (element by element): |O_gpu - O_oracle| <= 1e-2 (where |O_oracle| >= 4,
+where no bf16 number need lie within 1e-2 of the exact value, half a bf16 step
++ 1e-3), |LSE_gpu - LSE_oracle| <= 1e-3, -inf logsumexp exactly where the
+oracle has one, no NaN; the tile work list bit-exact against the CPU statement
+in oracle/schedule.py.
 """
 import numpy as np
 import pytest
@@ -268,6 +270,26 @@ def test_schedule_edge_lists_bit_exact():
         got = binding.varlen_attention_schedule(cq, ck, len(Lq), max(Lq), causal, W, cap)
         want = sch.schedule(workloads.cu_seqlens(Lq), workloads.cu_seqlens(Lk), causal, W)
         assert [tuple(r) for r in got.cpu().tolist()] == want
+
+
+@pytest.mark.parametrize("batch,seed", [(12000, 1), (21000, 2)])
+def test_schedule_bit_exact_beyond_one_sorted_run(batch, seed):
+    # more query blocks than one shared-memory sort holds (16384): runs sorted
+    # in shared memory, then merged in global memory (one merge pass, with the
+    # runs sorted in place, and two passes)
+    import random
+    from oracle import schedule as sch
+    rng = random.Random(seed)
+    Lq = [rng.randint(1, 700) for _ in range(batch)]
+    Lk = [x + rng.randint(0, 300) for x in Lq]
+    cu_q, cu_k = workloads.cu_seqlens(Lq), workloads.cu_seqlens(Lk)
+    cq = torch.tensor(cu_q, dtype=torch.int32, device="cuda")
+    ck = torch.tensor(cu_k, dtype=torch.int32, device="cuda")
+    cap = batch * ((max(Lq) + 255) // 256)
+    got = binding.varlen_attention_schedule(cq, ck, batch, max(Lq), True, 300, cap).cpu().numpy()
+    want = np.array(sch.schedule(cu_q, cu_k, True, 300), dtype=np.int32)
+    assert want.shape[0] > 16384
+    assert got.shape == want.shape and np.array_equal(got, want)
 
 
 def test_schedule_overflow_is_reported():

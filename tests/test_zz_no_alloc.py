@@ -5,26 +5,33 @@ serving runtime that owns all device memory through its own allocator, or a
 latency-critical loop that may not reach cudaMalloc or a stream-ordered
 allocator.  varlen_attention_fwd_noalloc serves them from a static per-device
 scratch array.  This file checks, through the C ABI, that two calls in a row
-give what varlen_attention_fwd gives (within the parity tolerances of the
-other tests), including after a call of another shape has left different
-contents in the shared array, and that an over-size problem is refused.
+give what varlen_attention_fwd gives and what the fp64 oracle gives (within
+the parity tolerances of the other tests), including after a call of another
+shape has left different contents in the shared array, that calls after the
+first one leave the device's free memory unchanged in a process that never
+used the allocating entry points, and that an over-size problem is refused.
 
 It is collected last on purpose, and it loads everything it needs itself, so
 it passes alone in a fresh process as well as after the other tests.
 """
+import os
+import subprocess
+import sys
+
 import numpy as np
 import pytest
 import torch
 
 from variable_length_flash_varlen_b200 import binding, workloads
+from tests._helpers import compare, oracle_all
 
 pytestmark = pytest.mark.gpu
 
 O_TOL, LSE_TOL = 1e-2, 1e-3
 
 
-def _inputs(wl):
-    q, k, v = workloads.make_qkv(wl, device="cuda")
+def _inputs(wl, host=None):
+    q, k, v = [t.cuda() for t in host] if host is not None else workloads.make_qkv(wl, device="cuda")
     cq = torch.tensor(wl.cu_q, dtype=torch.int32, device="cuda")
     ck = torch.tensor(wl.cu_k, dtype=torch.int32, device="cuda")
     return q, k, v, cq, ck
@@ -52,17 +59,56 @@ def _gpu():
 
 @pytest.mark.parametrize("name,scale", [("gqa_causal", 0.25), ("worked_example", 1.0),
                                         ("sliding_window", 1 / 8)])
-def test_noalloc_matches_default_entry_on_two_calls(name, scale):
+def test_noalloc_matches_default_entry_on_two_calls(oracle_lib, name, scale):
     wl = workloads.named(name, scale=scale)
-    q, k, v, cq, ck = _inputs(wl)
+    host = workloads.make_qkv(wl)
+    q, k, v, cq, ck = _inputs(wl, host)
     ref_out, ref_lse = binding.varlen_attention_fwd(q, k, v, cq, ck, *_args(wl))
+    ora_out, ora_lse = oracle_all(oracle_lib, wl, *host)
     for _ in range(2):
         out = torch.full_like(q, float("nan"))
         lse = torch.full((wl.total_q, wl.H), float("nan"), dtype=torch.float32, device="cuda")
         binding.varlen_attention_fwd_noalloc(q, k, v, cq, ck, *_args(wl), out, lse)
         torch.cuda.synchronize()
         _close(out, lse, ref_out, ref_lse)
+        compare(out, lse, ora_out, ora_lse)
     assert binding.device_status(clear=True) == 0
+
+
+# Run in a fresh process that never calls an allocating entry point, so that no
+# pool of the library holds reserved memory an allocation could hide in: after
+# the first (set-up) call, more calls must leave the device's free memory as
+# it was.  The outputs are allocated before the first call.
+_FREE_MEMORY_SCRIPT = r"""
+import sys, torch
+sys.path.insert(0, sys.argv[1])
+from variable_length_flash_varlen_b200 import binding, workloads
+wl = workloads.named("gqa_causal", scale=0.05)
+q, k, v = workloads.make_qkv(wl, device="cuda")
+cq = torch.tensor(wl.cu_q, dtype=torch.int32, device="cuda")
+ck = torch.tensor(wl.cu_k, dtype=torch.int32, device="cuda")
+out = torch.empty_like(q)
+lse = torch.empty(wl.total_q, wl.H, dtype=torch.float32, device="cuda")
+args = (wl.batch, wl.H, wl.H_kv, wl.max_seqlen_q, wl.max_seqlen_k, wl.D, wl.causal, wl.window)
+binding.varlen_attention_fwd_noalloc(q, k, v, cq, ck, *args, out, lse)
+torch.cuda.synchronize()
+free0 = torch.cuda.mem_get_info()[0]
+for _ in range(3):
+    binding.varlen_attention_fwd_noalloc(q, k, v, cq, ck, *args, out, lse)
+torch.cuda.synchronize()
+free1 = torch.cuda.mem_get_info()[0]
+print("FREE", free0, free1)
+"""
+
+
+def test_noalloc_calls_leave_free_device_memory_unchanged():
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _FREE_MEMORY_SCRIPT, root], capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = [x for x in r.stdout.splitlines() if x.startswith("FREE")][-1]
+    free0, free1 = (int(x) for x in line.split()[1:])
+    assert free0 == free1, f"free device memory moved from {free0} to {free1} bytes"
 
 
 def test_noalloc_serves_single_query_sequences():

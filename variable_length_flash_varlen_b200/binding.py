@@ -17,6 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libvarlen_attn.so")
 
 VA_OK = 0
+VA_ERR_INVALID_ARG, VA_ERR_UNSUPPORTED, VA_ERR_CUDA, VA_ERR_DEVICE_TIMEOUT = -1, -2, -3, -4
 VA_PATH_AUTO, VA_PATH_PREFILL, VA_PATH_DECODE = 0, 1, 2
 VA_STATUS_WAIT_TIMEOUT = 1
 VA_STATUS_SCHEDULE_OVERFLOW = 2
@@ -34,6 +35,7 @@ SIGNATURES = {
     "varlen_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_schedule": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P]),
     "varlen_attention_device_status": (_I, [ctypes.POINTER(ctypes.c_uint), _I]),
+    "varlen_attention_sync_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint), _I]),
     "varlen_attention_validate_cu_seqlens": (_I, [_P, _I, _I, _I, _I, _P]),
     "varlen_attention_selftest_wait_timeout": (_I, [_P, _P]),
     "varlen_attention_last_error": (ctypes.c_char_p, []),
@@ -305,6 +307,18 @@ def device_status(clear: bool = True) -> int:
     st = ctypes.c_uint(0)
     _check(load().varlen_attention_device_status(ctypes.byref(st), int(clear)))
     return st.value
+
+
+def sync_status(stream: Optional[torch.cuda.Stream] = None, clear: bool = True) -> Tuple[int, int]:
+    """Stream-scoped status query: (return code, status bits) once the work
+    enqueued on `stream` has finished.  The code is VA_OK, VA_ERR_DEVICE_TIMEOUT
+    (a bounded wait gave up) or VA_ERR_INVALID_ARG (schedule overflow); a CUDA
+    failure raises."""
+    st = ctypes.c_uint(0)
+    rc = load().varlen_attention_sync_status(_stream_ptr(stream), ctypes.byref(st), int(clear))
+    if rc == VA_ERR_CUDA:
+        _check(rc)
+    return rc, st.value
 
 
 def selftest_wait_timeout(stream: Optional[torch.cuda.Stream] = None) -> int:

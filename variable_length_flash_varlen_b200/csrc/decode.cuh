@@ -19,7 +19,9 @@
 // warps are merged and the split's (m, l, O) written out.
 //
 // The combine takes M = max m_s, L = sum 2^(m_s - M) l_s,
-// O = sum 2^(m_s - M) O_s / L and logsumexp = (M + log2 L) ln 2 — the same
+// O = sum 2^(m_s - M) O_s / N with N the same sum over the splits'
+// normalisers (row sums of P as rounded for the product), and logsumexp =
+// (M + log2 L) ln 2 — the same
 // rescaling the online softmax of realizar 0.8.4 attention.rs (IMP-111
 // online_softmax) applies tile by tile, applied once across splits.
 #pragma once
@@ -51,7 +53,7 @@ struct DecodeParams {
     const __nv_bfloat16* k;
     const __nv_bfloat16* v;
     float* part_o;   // [batch, H, n_split_max, D]
-    float* part_ml;  // [batch, H, n_split_max, 2]
+    float* part_ml;  // [batch, H, n_split_max, 4]: m, row sum of P, normaliser (rounded P's sum), -
     int* counter;    // unit counter, zero before the launch
     int n_split_max;
     int chunk;
@@ -72,8 +74,8 @@ struct DecodeSmem {
     static constexpr int kTileBytes = kDecodeTileKeys * D * 2;
     static constexpr int kK = 0;
     static constexpr int kV = kK + kStages * kTileBytes;
-    static constexpr int kRed = kV + kStages * kTileBytes;           // [warps][heads][D + 2] f32
-    static constexpr int kRedBytes = kDecodeComputeWarps * kDecodeHeads * (D + 2) * 4;
+    static constexpr int kRed = kV + kStages * kTileBytes;           // [warps][heads][D + 3] f32
+    static constexpr int kRedBytes = kDecodeComputeWarps * kDecodeHeads * (D + 3) * 4;
     static constexpr int kBar = kRed + kRedBytes;                    // full[S], empty[S], item_full[2], item_empty[2]
     static constexpr int kMisc = kBar + (2 * kStages + 4) * 8;
     static constexpr int kBytes = kMisc + 16;                        // abort flag, item ring[2]
@@ -90,7 +92,14 @@ __device__ __forceinline__ void decode_row_interval(const DecodeParams& p, int b
 
 struct DecodeUnit {
     int b, hk, g0, nh, split, k_begin, n_keys;
+    bool residual;  // the row sees few keys: P's bf16 rounding residual is multiplied in too
 };
+
+// A query that sees at most this many keys puts most of its softmax weight on
+// a few of them, and the bf16 rounding of P (2^-9 relative per weight) no
+// longer averages out; its units also multiply V by the residual
+// P - bf16(P), rounded to bf16 (two more tensor-core products per 16 keys).
+constexpr int kDecodeResidualMaxKeys = 256;
 
 // Unit u -> its sequence, head group and key range; false if it holds no key.
 __device__ __forceinline__ bool decode_unit(const DecodeParams& p, int u, DecodeUnit& w) {
@@ -108,6 +117,7 @@ __device__ __forceinline__ bool decode_unit(const DecodeParams& p, int u, Decode
     if (L_q <= 0 || hi < lo) return false;
     w.k_begin = lo + w.split * p.chunk;
     if (w.k_begin > hi) return false;
+    w.residual = hi - lo + 1 <= kDecodeResidualMaxKeys;
     w.n_keys = min(hi + 1, w.k_begin + p.chunk) - w.k_begin;
     return true;
 }
@@ -324,7 +334,9 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         float o[D / 8][4];
 #pragma unroll
         for (int nb = 0; nb < D / 8; ++nb) o[nb][0] = o[nb][1] = o[nb][2] = o[nb][3] = 0.f;
-        float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};   // rows g, g + 8
+        // rows g, g + 8: reference max, row sum of P, normaliser (sum of the P the
+        // product multiplies)
+        float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f}, ln[2] = {0.f, 0.f};
 
         const int n_tiles = (w.n_keys + kDecodeTileKeys - 1) / kDecodeTileKeys;
         bool ok = true;
@@ -374,6 +386,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                         m[r] = mt[r];
                     }
                     l[r] *= alpha[r];
+                    ln[r] *= alpha[r];
                 }
 #pragma unroll
                 for (int nb = 0; nb < D / 8; ++nb) {
@@ -393,16 +406,44 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                 pr[n][2] = ex2_approx(sc[n][2] - mu1);
                 pr[n][3] = ex2_approx(sc[n][3] - mu1);
             }
-            l[0] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
-            l[1] += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
             const uint32_t pa[4] = {pack_bf16x2(pr[0][0], pr[0][1]), pack_bf16x2(pr[0][2], pr[0][3]),
                                     pack_bf16x2(pr[1][0], pr[1][1]), pack_bf16x2(pr[1][2], pr[1][3])};
+            // bf16 bits are the upper half of the f32 bits
+            auto lo_of = [](uint32_t b2) { return __uint_as_float(b2 << 16); };
+            auto hi_of = [](uint32_t b2) { return __uint_as_float(b2 & 0xFFFF0000u); };
+            l[0] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+            l[1] += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
+            if (!w.residual) {
+                // the normaliser takes P as rounded to bf16, the values the PV product
+                // multiplies, so a dominant weight's rounding cancels in O / l; the
+                // logsumexp keeps the sum of P itself
+                ln[0] = add_bf16x2_f32(pa[2], add_bf16x2_f32(pa[0], ln[0]));
+                ln[1] = add_bf16x2_f32(pa[3], add_bf16x2_f32(pa[1], ln[1]));
 #pragma unroll
-            for (int db = 0; db < D / 16; ++db) {
-                uint32_t b[4];
-                ldsm_x4_trans(vt + (db >> 2) * L::kHalfBytes + offv[db & 3], b);
-                mma_16816(o[2 * db], pa, b[0], b[1]);
-                mma_16816(o[2 * db + 1], pa, b[2], b[3]);
+                for (int db = 0; db < D / 16; ++db) {
+                    uint32_t b[4];
+                    ldsm_x4_trans(vt + (db >> 2) * L::kHalfBytes + offv[db & 3], b);
+                    mma_16816(o[2 * db], pa, b[0], b[1]);
+                    mma_16816(o[2 * db + 1], pa, b[2], b[3]);
+                }
+            } else {
+                ln[0] += (pr[0][0] + pr[0][1]) + (pr[1][0] + pr[1][1]);
+                ln[1] += (pr[0][2] + pr[0][3]) + (pr[1][2] + pr[1][3]);
+                // f32 minus its bf16 rounding is exact
+                const uint32_t ra[4] = {
+                    pack_bf16x2(pr[0][0] - lo_of(pa[0]), pr[0][1] - hi_of(pa[0])),
+                    pack_bf16x2(pr[0][2] - lo_of(pa[1]), pr[0][3] - hi_of(pa[1])),
+                    pack_bf16x2(pr[1][0] - lo_of(pa[2]), pr[1][1] - hi_of(pa[2])),
+                    pack_bf16x2(pr[1][2] - lo_of(pa[3]), pr[1][3] - hi_of(pa[3]))};
+#pragma unroll
+                for (int db = 0; db < D / 16; ++db) {
+                    uint32_t b[4];
+                    ldsm_x4_trans(vt + (db >> 2) * L::kHalfBytes + offv[db & 3], b);
+                    mma_16816(o[2 * db], pa, b[0], b[1]);
+                    mma_16816(o[2 * db + 1], pa, b[2], b[3]);
+                    mma_16816(o[2 * db], ra, b[0], b[1]);
+                    mma_16816(o[2 * db + 1], ra, b[2], b[3]);
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
@@ -414,12 +455,14 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
         for (int r = 0; r < 2; ++r) {
             l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
             l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
+            ln[r] += __shfl_xor_sync(0xffffffffu, ln[r], 1);
+            ln[r] += __shfl_xor_sync(0xffffffffu, ln[r], 2);
         }
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             const int row = g + 8 * r;
             if (row < w.nh) {
-                float* dst = red + (warp * kDecodeHeads + row) * (D + 2);
+                float* dst = red + (warp * kDecodeHeads + row) * (D + 3);
 #pragma unroll
                 for (int nb = 0; nb < D / 8; ++nb) {
                     dst[nb * 8 + 2 * tq] = o[nb][2 * r];
@@ -428,6 +471,7 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
                 if (tq == 0) {
                     dst[D] = m[r];
                     dst[D + 1] = l[r];
+                    dst[D + 2] = ln[r];
                 }
             }
         }
@@ -437,20 +481,22 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_const
             float M = -INFINITY;
 #pragma unroll
             for (int ww = 0; ww < kDecodeComputeWarps; ++ww)
-                M = fmaxf(M, red[(ww * kDecodeHeads + hh) * (D + 2) + D]);
-            float acc = 0.f, lsum = 0.f;
+                M = fmaxf(M, red[(ww * kDecodeHeads + hh) * (D + 3) + D]);
+            float acc = 0.f, lsum = 0.f, nsum = 0.f;
 #pragma unroll
             for (int ww = 0; ww < kDecodeComputeWarps; ++ww) {
-                const float* src = red + (ww * kDecodeHeads + hh) * (D + 2);
+                const float* src = red + (ww * kDecodeHeads + hh) * (D + 3);
                 const float f = (src[D] == -INFINITY) ? 0.f : ex2_approx(src[D] - M);
                 acc = fmaf(src[d], f, acc);
                 lsum = fmaf(src[D + 1], f, lsum);
+                nsum = fmaf(src[D + 2], f, nsum);
             }
             const size_t slot = (static_cast<size_t>(w.b) * p.H + h0 + hh) * p.n_split_max + w.split;
             p.part_o[slot * D + d] = acc;
             if (d == 0) {
-                p.part_ml[slot * 2 + 0] = M;
-                p.part_ml[slot * 2 + 1] = lsum;
+                p.part_ml[slot * 4 + 0] = M;
+                p.part_ml[slot * 4 + 1] = lsum;
+                p.part_ml[slot * 4 + 2] = nsum;
             }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kDecodeComputeWarps) : "memory");
@@ -474,14 +520,15 @@ decode_combine_kernel(const DecodeParams p) {
     const int ns = (hi - lo + 1 + p.chunk - 1) / p.chunk;
     const size_t slot0 = (static_cast<size_t>(b) * p.H + h) * p.n_split_max;
     float M = -INFINITY;
-    for (int s = 0; s < ns; ++s) M = fmaxf(M, p.part_ml[(slot0 + s) * 2]);
-    float Lsum = 0.f, o = 0.f;
+    for (int s = 0; s < ns; ++s) M = fmaxf(M, p.part_ml[(slot0 + s) * 4]);
+    float Lsum = 0.f, Nsum = 0.f, o = 0.f;
     for (int s = 0; s < ns; ++s) {
-        const float w = ex2_approx(p.part_ml[(slot0 + s) * 2] - M);
-        Lsum = fmaf(w, p.part_ml[(slot0 + s) * 2 + 1], Lsum);
+        const float w = ex2_approx(p.part_ml[(slot0 + s) * 4] - M);
+        Lsum = fmaf(w, p.part_ml[(slot0 + s) * 4 + 1], Lsum);
+        Nsum = fmaf(w, p.part_ml[(slot0 + s) * 4 + 2], Nsum);
         o = fmaf(w, p.part_o[(slot0 + s) * D + d], o);
     }
-    p.out[out_row * D + d] = __float2bfloat16_rn(o / Lsum);
+    p.out[out_row * D + d] = __float2bfloat16_rn(o / Nsum);
     if (d == 0) p.lse[out_row] = (M + log2f(Lsum)) * 0.69314718055994530942f;
 }
 

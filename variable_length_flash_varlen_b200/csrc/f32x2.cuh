@@ -32,6 +32,16 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+// A packed bf16 pair (low half = first value) widened to an f32 pair:
+// the bf16 bits are the upper half of the f32 bits.
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t b2) {
+    return f2_pack(__uint_as_float(b2 << 16), __uint_as_float(b2 & 0xFFFF0000u));
+}
 // max of three (one instruction)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float r;

@@ -17,7 +17,8 @@
 //               shared memory (8-row boxes and one group of plain loads for
 //               a tile that runs past the end of the packed tensor)
 // Tensor memory (512 columns): S_0 at 0, S_1 at 128 (P_h aliases the first
-// 64 columns of S_h, or 32 for E4M3), O_0 at 256, O_1 at 256 + D.
+// 64 columns of S_h, or 32 for E4M3; the residual variant's P - bf16(P) the
+// next 64), O_0 at 256, O_1 at 256 + D.
 //
 // Two element formats share this code (the ElemBf16 / ElemE4m3 traits):
 // bf16 inputs and output (kind::f16 MMAs), and E4M3 inputs and output with
@@ -241,9 +242,15 @@ __device__ __forceinline__ void store_row_zero(const PrefillParams& p, size_t ou
     p.lse[out_row] = -INFINITY;
 }
 
-template <int D, class E>
+// kRes (bf16 only): the variant that serves the list's second part, the query
+// blocks holding a row that sees few keys, with every role's per-item code
+// also multiplying V by P's bf16 rounding residual (see kResidualMaxKeys); the
+// main variant carries none of that code.  The host launches the main variant,
+// then the residual variant as its programmatic dependent.
+template <int D, class E, bool kRes>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams p) {
+    static_assert(!(kRes && E::kFp8), "the residual variant is bf16 only");
     using L = PrefillSmem<D, E>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -299,15 +306,31 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
         prefetch_tensormap(&maps.k);
         prefetch_tensormap(&maps.v);
     }
-    // the set-up above overlaps the schedule build (programmatic dependent
-    // launch); everything below reads the list it writes
-    grid_dependency_wait();
+    if constexpr (!kRes) {
+        // The set-up above overlaps the schedule build (programmatic dependent
+        // launch); everything below reads the list it writes.  Once every CTA
+        // is past this wait the list is complete, and the residual variant,
+        // launched next, may start on the SMs this grid leaves as its work runs
+        // out (the list's second part is short).
+        grid_dependency_wait();
+        grid_launch_dependents();
+    }
+    // (The residual variant is launched only once every CTA of the main
+    // variant is past its wait for the schedule build, so the list is complete
+    // when it reads it; it waits for the main variant's completion before it
+    // exits, which keeps the stream's order for whatever follows.)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    const int n_items = min(max(p.hdr->n_tiles, 0), p.tile_capacity) * p.H;
+    // this variant's part of the list as item indices (block index x H +
+    // head): the main part [0, n_main H), the few-key part [n_main H, n_list H)
+    const int n_list = min(max(p.hdr->n_tiles, 0), p.tile_capacity);
+    const int n_main = min(max(p.hdr->n_main, 0), n_list);
+    const int item0 = kRes ? n_main * p.H : 0;
+    const int n_items = (kRes ? n_list - n_main : n_main) * p.H;
+    int* counter = kRes ? &p.hdr->next_item_res : &p.hdr->next_item;
     const int group = p.H / p.H_kv;
     unsigned* status = &g_va_status;
 
@@ -321,8 +344,8 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
             // claim the next work item (longest first across the grid) and publish it
             int idx = -1;
             if (lane == 0) {
-                const int t = atomicAdd(&p.hdr->next_item, 1);
-                idx = t < n_items ? t : -1;
+                const int t = atomicAdd(counter, 1);
+                idx = t < n_items ? item0 + t : -1;
             }
             idx = __shfl_sync(0xffffffffu, idx, 0);
             Item it;
@@ -438,6 +461,16 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                         mma_ts_lh<idesc_pv>(tmem + L::tmem_o(x), tmem + L::tmem_s(x) + kk * 8, vk,
                                             v_hi, acc);
                 }
+                if constexpr (kRes) {
+                    // the same keys' residual P - bf16(P), stored 64 columns further on
+#pragma unroll
+                    for (int k4 = 0; k4 < kSteps; ++k4) {
+                        const int kk = part * kSteps + k4;
+                        const uint32_t vk = vb + ((kk * kStepKeys * 128) >> 4);
+                        mma_ts_lh<idesc_pv>(tmem + L::tmem_o(x), tmem + L::tmem_s(x) + 64 + kk * 8,
+                                            vk, v_hi, 1u);
+                    }
+                }
                 if (last) mma_commit(&o_done[x]);
             };
 
@@ -546,7 +579,9 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
             // keys every row of this warp sees: tiles inside [warp_lo, warp_hi] need no mask
             const int warp_lo = __reduce_max_sync(0xffffffffu, lo);
             const int warp_hi = __reduce_min_sync(0xffffffffu, hi);
-            float m_ref = -INFINITY, l = 0.f;
+            // l: row sum of P (for the logsumexp); l_norm: the normaliser of O, the
+            // row sum of P as the PV product sees it (see the tile-maximum term below)
+            float m_ref = -INFINITY, l = 0.f, l_norm = 0.f;
             for (int kt = it.lo_h[x]; kt < it.hi_h[x]; ++kt) {
                 const bool first_tile = kt == it.lo_h[x];
                 if (!(ok = mbar_wait_warp(&s_full[x], s_waits++ & 1, abort_flag, status))) break;
@@ -603,6 +638,18 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                     m_ref = m_cand;
                 }
                 const float m_sub = (m_ref == -INFINITY) ? 0.f : m_ref;
+                // The PV product multiplies P as rounded to the input format, the row
+                // sum takes P itself; where one weight dominates a row, the dominant
+                // weight's rounding would then scale O by up to 2^-9.  So the
+                // normaliser also takes the rounding of each tile's largest P (the
+                // same FMA and exp2 the loop below applies to that score; 0 for a
+                // row that sees no key of the tile).  The residual variant multiplies
+                // P's rounding residual too, so there the normaliser is P's sum.
+                float tmax_round = 0.f;
+                if constexpr (!E::kFp8 && !kRes) {
+                    const float pt = ex2_approx(__fmaf_rn(mx, p.scale_log2, -m_sub));
+                    tmax_round = __bfloat162float(__float2bfloat16_rn(pt)) - pt;
+                }
                 // P = 2^(s * scale_log2 - m_ref) into S_x in the input format (bf16
                 // pairs or E4M3 quadruples), 64 keys at a time; the first 64 are handed over on their own so
                 // their PV starts while the second half is computed.  S_x's previous P
@@ -630,6 +677,31 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                             pk[c / 4] = pack_e4m3x4(p0, p1, p2, p3);
                         }
                         tmem_st16(sbase + half * 16, pk);
+                    } else if constexpr (kRes) {
+                        // P as bf16 plus its residual P - bf16(P) (exact in f32) as bf16,
+                        // 64 columns further on, over scores already read; 16 keys at a
+                        // time
+#pragma unroll
+                        for (int q8 = 0; q8 < 4; ++q8) {
+                            const int k0 = half * 64 + q8 * 16;
+                            uint32_t pk[8], rk[8];
+#pragma unroll
+                            for (int c = 0; c < 16; c += 2) {
+                                float x0, x1;
+                                f2_unpack(f2_fma(f2_pack(s[k0 + c], s[k0 + c + 1]), scale2, neg2), x0, x1);
+                                const uint64_t pp = f2_pack(ex2_approx(x0), ex2_approx(x1));
+                                sum2[(c >> 1) & 3] = f2_add(sum2[(c >> 1) & 3], pp);
+                                float p0, p1;
+                                f2_unpack(pp, p0, p1);
+                                const uint32_t b2 = pack_bf16x2(p0, p1);
+                                pk[c / 2] = b2;
+                                float r0, r1;
+                                f2_unpack(f2_sub(pp, bf16x2_to_f2(b2)), r0, r1);
+                                rk[c / 2] = pack_bf16x2(r0, r1);
+                            }
+                            tmem_st8(sbase + half * 32 + q8 * 8, pk);
+                            tmem_st8(sbase + 64 + half * 32 + q8 * 8, rk);
+                        }
                     } else {
                         uint32_t pk[32];
 #pragma unroll
@@ -668,8 +740,10 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
                 float sums[8];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) f2_unpack(sum2[e], sums[2 * e], sums[2 * e + 1]);
-                l = l * alpha + (((sums[0] + sums[1]) + (sums[2] + sums[3])) +
-                                 ((sums[4] + sums[5]) + (sums[6] + sums[7])));
+                const float tile_sum = ((sums[0] + sums[1]) + (sums[2] + sums[3])) +
+                                       ((sums[4] + sums[5]) + (sums[6] + sums[7]));
+                l = l * alpha + tile_sum;
+                l_norm = l_norm * alpha + (tile_sum + tmax_round);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -682,7 +756,7 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
             tc_fence_after();
             // O / l, times v_scale / o_scale for E4M3 (V's dequantization and the
             // output's quantization folded into one factor)
-            const float inv_l = l > 0.f ? p.out_mul / l : 0.f;
+            const float inv_l = l_norm > 0.f ? p.out_mul / l_norm : 0.f;
             {
                 // every column block in flight before a single wait
                 uint32_t r[D / 32][32];
@@ -746,6 +820,7 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    if constexpr (kRes) grid_dependency_wait();
 }
 
 }  // namespace va

@@ -245,6 +245,13 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -349,6 +356,16 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float b0, float b1, float b2, fl
         : "=r"(r)
         : "f"(b0), "f"(b1), "f"(b2), "f"(b3));
     return r;
+}
+
+// acc + both values of a packed bf16 pair, each widened exactly to f32
+// (mixed-precision adds, one rounding each).
+__device__ __forceinline__ float add_bf16x2_f32(uint32_t b2, float acc) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %0, hi, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(b2));
+    return acc;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

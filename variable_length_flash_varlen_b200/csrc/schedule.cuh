@@ -79,11 +79,38 @@ __host__ __device__ __forceinline__ void rows_key_range(int first, int rows, int
     kt_hi = hi1 / kBlockN + 1;
 }
 
+// A row that sees at most this many keys puts most of its softmax weight on a
+// few of them, and there the bf16 rounding of P (2^-9 relative per weight) no
+// longer averages out: its output can move by ~2^-9 |v|, beyond what a bf16
+// result may differ from the exact one.  Query blocks holding such a row are
+// listed apart and run by a kernel variant that also multiplies V by the
+// residual P - bf16(P), rounded to bf16 (~2^-17 relative).
+constexpr int kResidualMaxKeys = 256;
+
+// Does some row of [first, first + rows) (clipped to L_q) see between 1 and
+// kResidualMaxKeys keys?  The visible count of a row never decreases with the
+// row index (the band's upper end moves with the diagonal, its width is
+// fixed), so the first row that sees any key has the fewest.
+__host__ __device__ __forceinline__ bool rows_see_few_keys(int first, int rows, int L_q, int L_k,
+                                                           bool causal, int window) {
+    int i0 = first;
+    if ((causal || window > 0) && L_q - L_k > i0) i0 = L_q - L_k;
+    const int end = L_q < first + rows ? L_q : first + rows;
+    if (i0 >= end) return false;
+    int lo, hi;
+    row_key_interval(i0, L_q, L_k, causal, window, lo, hi);
+    return hi >= lo && hi - lo + 1 <= kResidualMaxKeys;
+}
+
 // Workspace header written by the builder and read by the attention kernels.
+// The list holds n_main blocks first, then n_tiles - n_main blocks that hold a
+// row seeing few keys (each part longest first); each part has its own work
+// counter, claimed by its own kernel variant.
 struct SchedHeader {
-    int n_tiles;    // number of valid entries in the sorted list
-    int next_item;  // work counter of the persistent grid (zeroed by the builder)
-    int pad[2];
+    int n_tiles;        // number of valid entries in the sorted list
+    int next_item;      // work counter over the first part (zeroed by the builder)
+    int n_main;         // entries of the first part
+    int next_item_res;  // work counter over the second part (zeroed by the builder)
 };
 
 }  // namespace va

@@ -66,6 +66,26 @@ constexpr int kMaxDevices = 64;
 constexpr int kHostChunks = 4;
 constexpr size_t kHostChunkMinBytes = size_t(8) << 20;
 
+// Shared-memory limits of every prefill kernel variant.
+int set_prefill_attributes() {
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<64, va::ElemBf16, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::PrefillSmem<64, va::ElemBf16>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<64, va::ElemBf16, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::PrefillSmem<64, va::ElemBf16>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128, va::ElemBf16, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::PrefillSmem<128, va::ElemBf16>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128, va::ElemBf16, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::PrefillSmem<128, va::ElemBf16>::kAlloc));
+    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128, va::ElemE4m3, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::PrefillSmem<128, va::ElemE4m3>::kAlloc));
+    return VA_OK;
+}
+
 struct DeviceInfo {
     bool ready = false;
     int num_sms = 0;
@@ -100,15 +120,7 @@ int device_setup(int& dev, DeviceInfo*& info) {
             return fail(VA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
         g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<64, va::ElemBf16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::PrefillSmem<64, va::ElemBf16>::kAlloc));
-    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128, va::ElemBf16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::PrefillSmem<128, va::ElemBf16>::kAlloc));
-    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128, va::ElemE4m3>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::PrefillSmem<128, va::ElemE4m3>::kAlloc));
+    if (set_prefill_attributes() != VA_OK) return VA_ERR_CUDA;
     VA_CUDA(cudaFuncSetAttribute(va::build_schedule_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  va::kSortCapacity * 8));
@@ -172,6 +184,29 @@ int make_tile_map(CUtensorMap* map, const void* base, long long cols, long long 
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The packed layout's preconditions on one host cu_seqlens array (boostr
+// varlen_attention.rs, VarLenAttentionOps docs, "Layout contract": cumulative
+// lengths starting at 0): c[0] == 0, never decreasing, no step above
+// max_seqlen and, when total >= 0, c[batch] == total.  Reads entries
+// 0..batch only.
+int check_cu_seqlens_host(const int32_t* c, int batch, int max_seqlen, long long total,
+                          const char* name) {
+    if (c[0] != 0) return fail(VA_ERR_INVALID_ARG, "%s[0] = %d, must be 0", name, c[0]);
+    for (int b = 0; b < batch; ++b) {
+        const long long len = static_cast<long long>(c[b + 1]) - c[b];
+        if (len < 0)
+            return fail(VA_ERR_INVALID_ARG, "%s decreases at entry %d (%d -> %d)", name, b + 1,
+                        c[b], c[b + 1]);
+        if (len > max_seqlen)
+            return fail(VA_ERR_INVALID_ARG, "sequence %d has length %lld > max_seqlen %d (%s)", b,
+                        len, max_seqlen, name);
+    }
+    if (total >= 0 && c[batch] != total)
+        return fail(VA_ERR_INVALID_ARG, "%s[%d] = %d, expected the total %lld", name, batch,
+                    c[batch], total);
+    return VA_OK;
+}
 
 struct Args {
     const void *q, *k, *v;
@@ -282,14 +317,22 @@ cudaError_t launch_prefill(const Args& a, const va::PrefillMaps& maps, const va:
     cfg.numAttrs = 1;
     if (a.fp8) {
         cfg.dynamicSmemBytes = va::PrefillSmem<128, va::ElemE4m3>::kAlloc;
-        return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<128, va::ElemE4m3>, maps, p);
+        return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<128, va::ElemE4m3, false>, maps, p);
     }
+    // bf16: the main variant over the list's main part, then the residual
+    // variant over its few-key part, a programmatic dependent launch of the
+    // main one that starts on the SMs the main one leaves as its work runs out
+    cudaError_t e;
     if (a.D == 64) {
         cfg.dynamicSmemBytes = va::PrefillSmem<64, va::ElemBf16>::kAlloc;
-        return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<64, va::ElemBf16>, maps, p);
+        e = cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<64, va::ElemBf16, false>, maps, p);
+        if (e != cudaSuccess) return e;
+        return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<64, va::ElemBf16, true>, maps, p);
     }
     cfg.dynamicSmemBytes = va::PrefillSmem<128, va::ElemBf16>::kAlloc;
-    return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<128, va::ElemBf16>, maps, p);
+    e = cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<128, va::ElemBf16, false>, maps, p);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<128, va::ElemBf16, true>, maps, p);
 }
 
 int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
@@ -316,7 +359,8 @@ int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
     }
 
     va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
-        a.cu_q, a.cu_k, a.seqused_k, a.batch, a.causal, a.window, cap, key_slots, scratch, tiles, hdr);
+        a.cu_q, a.cu_k, a.seqused_k, a.batch, a.causal, a.window, a.fp8 ? 0 : 1, cap, key_slots,
+        scratch, tiles, hdr);
     cudaError_t be = cudaGetLastError();
     if (be != cudaSuccess) {
         cudaFreeAsync(ws, stream);
@@ -356,7 +400,7 @@ int run_decode(const Args& a, const DeviceInfo& dev, int split_keys, cudaStream_
     const size_t hdr = 256;
     const size_t o_bytes = slots * a.D * sizeof(float);
     char* ws = nullptr;
-    VA_CUDA(ws_alloc(reinterpret_cast<void**>(&ws), hdr + o_bytes + slots * 2 * sizeof(float), stream));
+    VA_CUDA(ws_alloc(reinterpret_cast<void**>(&ws), hdr + o_bytes + slots * 4 * sizeof(float), stream));
     cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int), stream);
     if (e != cudaSuccess) {
         cudaFreeAsync(ws, stream);
@@ -568,15 +612,7 @@ int noalloc_setup(NoAllocState*& st) {
             return fail(VA_ERR_CUDA, "cuTensorMapEncodeTiled entry point not found");
         g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<64, va::ElemBf16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::PrefillSmem<64, va::ElemBf16>::kAlloc));
-    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128, va::ElemBf16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::PrefillSmem<128, va::ElemBf16>::kAlloc));
-    VA_CUDA(cudaFuncSetAttribute(va::prefill_fwd_kernel<128, va::ElemE4m3>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::PrefillSmem<128, va::ElemE4m3>::kAlloc));
+    if (set_prefill_attributes() != VA_OK) return VA_ERR_CUDA;
     VA_CUDA(cudaFuncSetAttribute(va::build_schedule_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  va::kSortCapacity * 8));
@@ -615,7 +651,8 @@ int run_prefill_noalloc(const Args& a, cudaStream_t stream) {
     // the builder rewrites the whole header (count and work counter) and every
     // list entry it hands out, so nothing left by the previous call is read
     va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
-        a.cu_q, a.cu_k, a.seqused_k, a.batch, a.causal, a.window, cap, key_slots, scratch, tiles, hdr);
+        a.cu_q, a.cu_k, a.seqused_k, a.batch, a.causal, a.window, a.fp8 ? 0 : 1, cap, key_slots,
+        scratch, tiles, hdr);
     cudaError_t be = cudaGetLastError();
     if (be != cudaSuccess) return cuda_fail(be, "schedule build launch");
 
@@ -707,12 +744,16 @@ int varlen_attention_fwd_host(const void* q, const void* k, const void* v,
     int rc = validate(a);
     if (rc != VA_OK) return rc;
     if (batch == 0 || max_seqlen_q == 0) return VA_OK;
+    // The host arrays size every copy and every chunk below: check them before
+    // any device work (a decreasing entry would give negative offsets).
+    if ((rc = check_cu_seqlens_host(cu_seqlens_q, batch, max_seqlen_q, -1, "cu_seqlens_q")) != VA_OK ||
+        (rc = check_cu_seqlens_host(cu_seqlens_k, batch, max_seqlen_k, -1, "cu_seqlens_k")) != VA_OK)
+        return rc;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     int dev;
     DeviceInfo* info;
     if ((rc = device_setup(dev, info)) != VA_OK) return rc;
     const long long T_q = cu_seqlens_q[batch], T_k = cu_seqlens_k[batch];
-    if (T_q < 0 || T_k < 0) return fail(VA_ERR_INVALID_ARG, "negative total length");
     const size_t q_row = static_cast<size_t>(num_heads) * head_dim * 2;
     const size_t k_row = static_cast<size_t>(num_kv_heads) * head_dim * 2;
     const size_t l_row = static_cast<size_t>(num_heads) * 4;
@@ -861,7 +902,7 @@ int varlen_attention_schedule(const int32_t* cu_seqlens_q, const int32_t* cu_seq
     VA_CUDA(ws_alloc(reinterpret_cast<void**>(&ws), 256 + list_bytes, stream));
     auto* hdr = reinterpret_cast<va::SchedHeader*>(ws);
     va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
-        cu_seqlens_q, cu_seqlens_k, nullptr, batch, causal ? 1 : 0, window, capacity, key_slots,
+        cu_seqlens_q, cu_seqlens_k, nullptr, batch, causal ? 1 : 0, window, 1, capacity, key_slots,
         reinterpret_cast<va::TileEntry*>(ws + 256), reinterpret_cast<va::TileEntry*>(tiles), hdr);
     cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess)
@@ -887,20 +928,7 @@ int varlen_attention_validate_cu_seqlens(const int32_t* cu_seqlens, int batch, i
         VA_CUDA(cudaStreamSynchronize(stream));
         c = host.data();
     }
-    if (c[0] != 0) return fail(VA_ERR_INVALID_ARG, "cu_seqlens[0] = %d, must be 0", c[0]);
-    for (int b = 0; b < batch; ++b) {
-        const long long len = static_cast<long long>(c[b + 1]) - c[b];
-        if (len < 0)
-            return fail(VA_ERR_INVALID_ARG, "cu_seqlens decreases at entry %d (%d -> %d)", b + 1,
-                        c[b], c[b + 1]);
-        if (len > max_seqlen)
-            return fail(VA_ERR_INVALID_ARG, "sequence %d has length %lld > max_seqlen %d", b, len,
-                        max_seqlen);
-    }
-    if (total >= 0 && c[batch] != total)
-        return fail(VA_ERR_INVALID_ARG, "cu_seqlens[%d] = %d, expected the total %d", batch,
-                    c[batch], total);
-    return VA_OK;
+    return check_cu_seqlens_host(c, batch, max_seqlen, total, "cu_seqlens");
 }
 
 int varlen_attention_device_status(unsigned* status, int clear) {
@@ -912,6 +940,30 @@ int varlen_attention_device_status(unsigned* status, int clear) {
         const unsigned zero = 0;
         VA_CUDA(cudaMemcpyToSymbol(va::g_va_status, &zero, sizeof(unsigned)));
     }
+    return VA_OK;
+}
+
+int varlen_attention_sync_status(void* stream_, unsigned* status, int clear) {
+    g_last_error[0] = 0;
+    if (!status) return fail(VA_ERR_INVALID_ARG, "status is NULL");
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    unsigned word = 0;
+    VA_CUDA(cudaMemcpyFromSymbolAsync(&word, va::g_va_status, sizeof(unsigned), 0,
+                                      cudaMemcpyDeviceToHost, stream));
+    if (clear) {
+        // after the copy in the same stream's order
+        void* addr = nullptr;
+        VA_CUDA(cudaGetSymbolAddress(&addr, va::g_va_status));
+        VA_CUDA(cudaMemsetAsync(addr, 0, sizeof(unsigned), stream));
+    }
+    VA_CUDA(cudaStreamSynchronize(stream));
+    *status = word;
+    if (word & va::kStatusWaitTimeout)
+        return fail(VA_ERR_DEVICE_TIMEOUT, "a bounded wait inside a kernel gave up (status 0x%x)", word);
+    if (word & va::kStatusScheduleOverflow)
+        return fail(VA_ERR_INVALID_ARG,
+                    "more query blocks than max_seqlen_q allows for: a query length exceeds "
+                    "max_seqlen_q (status 0x%x)", word);
     return VA_OK;
 }
 
