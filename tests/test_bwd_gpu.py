@@ -130,15 +130,26 @@ def test_bwd_argument_errors():
     assert lib.varlen_attention_bwd(*ptrs, 1, 2, 1, 10, 10, 96, 0, 0, *outs) == -2
 
 
-def test_bwd_full_size_sampled_sequences(oracle_lib):
-    # the benchmark's backward workload in its launch configuration; sequences
-    # are independent, so the oracle on a few of them alone gives their exact
-    # gradients (the three shortest, to keep the fp64 run short)
-    wl = workloads.named("mha_noncausal")
+@pytest.mark.parametrize("name,pick", [("mha_noncausal", "shortest"), ("mha_noncausal", "longest"),
+                                       ("gqa_causal", "long")])
+def test_bwd_full_size_sampled_sequences(oracle_lib, name, pick):
+    # the benchmark's backward workloads in their launch configuration;
+    # sequences are independent, so the oracle on a few of them alone gives
+    # their exact gradients: the three shortest and the three longest of the
+    # MHA workload (the longest have the most key tiles per query tile), and one
+    # GQA causal sequence of at least 4096 tokens
+    wl = workloads.named(name)
     q, k, v = workloads.make_qkv(wl)
     do = _dout(wl, 7)
     gq, gk, gv = run_bwd(wl, q, k, v, do)
-    for b in sorted(range(wl.batch), key=lambda x: wl.lengths_q[x])[:3]:
+    order = sorted(range(wl.batch), key=lambda x: wl.lengths_q[x])
+    if pick == "shortest":
+        chosen = order[:3]
+    elif pick == "longest":
+        chosen = order[-3:]
+    else:
+        chosen = [next(b for b in order if wl.lengths_q[b] >= 4096)]
+    for b in chosen:
         q0, q1, k0, k1 = wl.cu_q[b], wl.cu_q[b + 1], wl.cu_k[b], wl.cu_k[b + 1]
         sub = workloads.custom([q1 - q0], [k1 - k0], wl.H, wl.H_kv, wl.D, wl.causal, wl.window,
                                seed=0)

@@ -138,9 +138,11 @@ def test_fp8_exact_p_leaves_only_output_rounding(oracle_lib, causal, W):
     compare_fp8(oracle_lib, out, lse, ref_o, ref_l, err, sc["o_scale"], p_exact=True)
 
 
-def test_fp8_full_size_sampled_rows(oracle_lib):
-    # the workload the benchmark times in FP8, in the same launch configuration
-    wl = workloads.named("mha_noncausal")
+@pytest.mark.parametrize("name", ["mha_noncausal", "gqa_causal", "sliding_window"])
+def test_fp8_full_size_sampled_rows(oracle_lib, name):
+    # full-size workloads in FP8 in the launch configuration the benchmark uses
+    # (the MHA one is the one it times)
+    wl = workloads.named(name)
     q8, k8, v8, sc = workloads.make_qkv_fp8(wl)
     out, lse = run_fp8(wl, q8, k8, v8, sc)
     rng = np.random.default_rng(5)
