@@ -19,8 +19,8 @@
  *     window_size W > 0 a query sees only the W most recent key positions;
  *     logsumexp is F32 and is what the backward pass consumes.
  *
- * Readings taken where the pages are silent (each one is listed in the
- * design notes of this repository):
+ * Readings taken where the pages are silent (the varlen trait defines no
+ * causal offset, window inclusivity, logsumexp base or empty-row result):
  *   - causal with L_q != L_k is bottom-right aligned: key j is visible to
  *     query i iff j <= i + (L_k - L_q);
  *   - the window holds exactly W keys ending at the diagonal:

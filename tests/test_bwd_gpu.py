@@ -3,7 +3,9 @@
 The GPU backward consumes the GPU forward's output and logsumexp (as the
 trait's varlen_attention_bwd does), rounds P and dS to bf16 for its tensor-core
 products and writes bf16 gradients; the oracle differentiates the exact
-attention of the same bf16 inputs in fp64.  Bar per tensor (reading r18):
+attention of the same bf16 inputs in fp64.  The trait's backward (boostr
+varlen_attention.rs, VarLenAttentionOps::varlen_attention_bwd) states no
+tolerance; the bar per tensor is:
 
   |g_gpu - g_ref| <= half a bf16 step at g_ref + 1e-2 * max |g_ref|
 
