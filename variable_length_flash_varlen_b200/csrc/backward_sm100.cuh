@@ -9,19 +9,25 @@
 //   dS_ij = P_ij (dP_ij - Delta_i)
 //   dv_j = sum_i P_ij dout_i,  dk_j = sum_i dS_ij q_i / sqrt(D),
 //   dq_i = sum_j dS_ij k_j / sqrt(D).
-// Two kernels, no atomics, every output element written by one CTA, dQ first:
-//   bwd_dq_kernel      one CTA per (128-row query tile, query head, sequence):
+// Two persistent kernels, no atomics, every output element written by one
+// CTA, dQ first.  Each works through a device-built list of its tiles,
+// longest first, claimed from a grid-wide counter (one CTA per SM):
+//   bwd_dq_kernel      item = (128-row query tile, query head, sequence):
 //                      Delta_i of its rows (stored for the other kernel), then
 //                      with Q and dout resident, for every visible key tile
 //                      S = Q K^T, dP = dout V^T, dS (bf16) into tensor memory,
 //                      dQ += dS K
-//   bwd_dkdv_kernel    one CTA per (key tile of 128 keys, KV head, sequence):
+//   bwd_dkdv_kernel    item = (key tile of 128 keys, KV head, sequence):
 //                      K and V stay in shared memory; for every query head of
 //                      the group and every 128-row query tile that sees the key
 //                      tile: S^T = K Q^T, then P^T (bf16) into tensor memory
 //                      while dP^T = V dout^T runs, then dS^T (bf16) while
 //                      dV += P^T dout runs, then dK += dS^T Q (TS form), the
 //                      two accumulators in tensor memory over the whole loop
+// An item's resident tiles are reloaded once its last products that read them
+// are done, its accumulators read out by the element-wise warps before the
+// next item's first product overwrites them; the products of one item's steps
+// and the barrier phases run on across items.
 // Warp roles (320 threads): warps 0-7 the element-wise work and the epilogue
 // (one key row, or one query row, per thread; warps w and w + 4 share a
 // tensor-memory lane quarter and take one half of the 128 columns each), warp
@@ -66,6 +72,21 @@ struct BwdParams {
     uint8_t* dv;
     float scale_log2;     // log2(e) / sqrt(D)
     float scale;          // 1 / sqrt(D)
+    // work lists (build_bwd_list_kernel): query tiles for dQ, key tiles for dK/dV
+    const TileEntry* list_q;
+    SchedHeader* hdr_q;
+    int cap_q;
+    const TileEntry* list_k;
+    SchedHeader* hdr_k;
+    int cap_k;
+};
+
+// A claimed work item as the producer publishes it to the other roles.
+struct BwdItem {
+    int idx;                // item index (entry x heads + head), -1 = no more work
+    int b, tile, a0, a1;    // the list entry
+    int head;
+    int pad[2];
 };
 
 // Q and dout as [rows][H * D], K and V as [rows][H_kv * D]: 128-row boxes and
@@ -88,10 +109,11 @@ struct BwdSmem {
     static constexpr int kRows = 6 * kTile;       // [2][128] f32 lse * log2(e), [2][128] f32 Delta
     static constexpr int kBar = kRows + 4 * 128 * 4;
     // fixed_full, ring_full[2], ring_empty[2], s_full, p_ready, acc_done, dp_full, ds_ready,
-    // p_read
-    static constexpr int kNumBars = 11;
+    // p_read, fixed_empty, acc_free, item_full[2], item_empty[2]
+    static constexpr int kNumBars = 17;
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag
-    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kItems = kMisc + 16;          // BwdItem [2]
+    static constexpr int kBytes = kItems + 2 * 32;
     static constexpr int kAlloc = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
     static_assert(kAlloc <= 232448, "beyond the 227 KB of shared memory a CTA may use");
 };
@@ -107,8 +129,13 @@ struct BwdBars {
     uint64_t* dp_full;   // dK/dV kernel: dP^T ready (S^T has its own s_full)
     uint64_t* ds_ready;  // dK/dV kernel: dS^T stored
     uint64_t* p_read;    // dK/dV kernel: the element-wise warps have loaded P^T (S^T may be overwritten)
+    uint64_t* fixed_empty;  // the item's last products that read the resident tiles are done
+    uint64_t* acc_free;     // the element-wise warps have read the item's accumulators out
+    uint64_t* item_full;    // [2]
+    uint64_t* item_empty;   // [2]
     uint32_t* tmem_slot;
     volatile int* abort_flag;
+    BwdItem* items;         // [2]
 };
 
 template <int D>
@@ -125,8 +152,13 @@ __device__ __forceinline__ BwdBars bwd_setup(uint8_t* smem, int warp) {
     r.dp_full = bars + 8;
     r.ds_ready = bars + 9;
     r.p_read = bars + 10;
+    r.fixed_empty = bars + 11;
+    r.acc_free = bars + 12;
+    r.item_full = bars + 13;
+    r.item_empty = bars + 15;
     r.tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     r.abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+    r.items = reinterpret_cast<BwdItem*>(smem + L::kItems);
     if (threadIdx.x == 0) {
         mbar_init(r.fixed_full, 2);  // two tile loads
         for (int s = 0; s < 2; ++s) {
@@ -139,6 +171,12 @@ __device__ __forceinline__ BwdBars bwd_setup(uint8_t* smem, int warp) {
         mbar_init(r.dp_full, 1);
         mbar_init(r.ds_ready, kBwdEwWarps);
         mbar_init(r.p_read, kBwdEwWarps);
+        mbar_init(r.fixed_empty, 1);
+        mbar_init(r.acc_free, kBwdEwWarps);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&r.item_full[s], 1);
+            mbar_init(&r.item_empty[s], 1 + kBwdEwWarps);  // the MMA lane and the element-wise warps
+        }
         *r.abort_flag = 0;
         fence_barrier_init();
     }
@@ -198,7 +236,8 @@ __device__ __forceinline__ void bwd_store_rows(uint32_t taddr, float mul, uint8_
 }
 
 // ---------------------------------------------------------------------------
-// dK, dV: one CTA per (key tile kt, KV head hk, sequence b) = blockIdx (x, y, z).
+// dK, dV: items (key tile kt, KV head hk, sequence b) from the list of key
+// tiles, longest first.
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
@@ -208,83 +247,102 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kt = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
     const int G = p.H / p.H_kv;
-    const int cq = p.cu_q[b], ck = p.cu_k[b];
-    const int L_q = p.cu_q[b + 1] - cq, L_k = p.cu_k[b + 1] - ck;
-    const int k0 = kt * kBlockN;
-    if (k0 >= L_k) return;  // the whole CTA, before any barrier
-    const int k_last = min(L_k, k0 + kBlockN) - 1;
-    const int delta_k = L_k - L_q;
-    // query rows that see a key of [k0, k_last] (bottom-right causal, window of
-    // W keys ending at the diagonal): i >= k0 - delta_k, i <= k_last - delta_k + W - 1
-    int r0 = 0, r1 = L_q - 1;
-    if (p.causal || p.window > 0) r0 = max(0, k0 - delta_k);
-    if (p.window > 0) r1 = min(r1, k_last - delta_k + p.window - 1);
-    const int n_qt = (L_q > 0 && r1 >= r0) ? r1 / kBlockM - r0 / kBlockM + 1 : 0;
-    const int qt0 = r0 / kBlockM;
-    const int n_steps = G * n_qt;
     const long long kv_pitch = static_cast<long long>(p.H_kv) * D * 2;
-    if (n_steps == 0) {
-        // no query sees these keys: their gradients are zero
-        for (int idx = threadIdx.x; idx < (k_last - k0 + 1) * (D / 8); idx += blockDim.x) {
-            const int r = idx / (D / 8), c = idx % (D / 8);
-            const long long off = (static_cast<long long>(ck) + k0 + r) * kv_pitch + hk * D * 2 + c * 16;
-            *reinterpret_cast<uint4*>(p.dk + off) = make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(p.dv + off) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        return;
-    }
-
     const BwdBars bar = bwd_setup<D>(smem, warp);
     const uint32_t tmem = *bar.tmem_slot;
     unsigned* status = &g_va_status;
     float* lse_s = reinterpret_cast<float*>(smem + L::kRows);            // [2][128]
     float* dlt_s = reinterpret_cast<float*>(smem + L::kRows + 1024);     // [2][128]
     constexpr uint32_t kS = 0, kDP = 128, kDV = 256, kDK = 256 + D;      // tensor-memory columns
+    const int n_items = min(max(p.hdr_k->n_tiles, 0), p.cap_k) * p.H_kv;
+    // An item's query rows that see one of its keys ([r0, r1], key_tile_rows)
+    // come in n_qt 128-row tiles from qt0; its steps are the G query heads x
+    // those tiles.
+    auto item_rows = [&](const BwdItem& it, int& qt0, int& n_qt) {
+        const int L_q = p.cu_q[it.b + 1] - p.cu_q[it.b], L_k = p.cu_k[it.b + 1] - p.cu_k[it.b];
+        int r0, r1;
+        key_tile_rows(it.tile, L_q, L_k, p.causal != 0, p.window, r0, r1);
+        qt0 = r0 / kBlockM;
+        n_qt = it.a1;
+    };
 
     if (warp == kBwdLoadWarp) {
         // ------------------------------------------------------------ producer
         const int T_q = p.cu_q[p.batch], T_k = p.cu_k[p.batch];
         const int q_stride = p.H * D * 2, kv_stride = p.H_kv * D * 2;
-        uint32_t issued[2] = {0, 0};
+        uint32_t ring_n = 0, fixed_n = 0, item_n = 0, issued[2] = {0, 0};
         bool ok = true;
-        load_tile<D, ElemBf16>(smem + L::kFixed0, &maps.k, &maps.k8, p.k, ck + k0, T_k, kv_stride,
-                               hk * D, bar.fixed_full, lane);
-        load_tile<D, ElemBf16>(smem + L::kFixed1, &maps.v, &maps.v8, p.v, ck + k0, T_k, kv_stride,
-                               hk * D, bar.fixed_full, lane);
-        for (int n = 0; n < n_steps; ++n) {
-            const int st = n & 1;
-            const int h = hk * G + n / n_qt, qt = qt0 + n % n_qt;
-            if (!(ok = mbar_wait_warp(&bar.ring_empty[st], ((n >> 1) & 1) ^ 1, bar.abort_flag, status)))
+        for (;;) {
+            int idx = -1;
+            if (lane == 0) {
+                const int t = atomicAdd(&p.hdr_k->next_item, 1);
+                idx = t < n_items ? t : -1;
+            }
+            idx = __shfl_sync(0xffffffffu, idx, 0);
+            BwdItem it{idx, 0, 0, 0, 0, 0, {0, 0}};
+            if (idx >= 0) {
+                const TileEntry e = p.list_k[idx / p.H_kv];
+                it = BwdItem{idx, e.b, e.qt, e.kt_lo, e.kt_hi, idx % p.H_kv, {0, 0}};
+            }
+            const int slot = item_n & 1;
+            if (!(ok = mbar_wait_warp(&bar.item_empty[slot], ((item_n >> 1) & 1) ^ 1, bar.abort_flag, status)))
                 break;
-            {
-                // the tile's 128 rows of {lse * log2(e), Delta}, staged negated (the
-                // element-wise warps add them): four loads per lane in flight at once
-                // (rows past the sequence are masked: any finite value)
-                const float2* src = p.rowinfo + h * p.rows_cap + cq + qt * kBlockM;
-                float2 ri[kBlockM / 32];
-#pragma unroll
-                for (int u = 0; u < kBlockM / 32; ++u) {
-                    const int r = lane + 32 * u;
-                    ri[u] = qt * kBlockM + r < L_q ? src[r] : make_float2(0.f, 0.f);
-                }
-#pragma unroll
-                for (int u = 0; u < kBlockM / 32; ++u) {
-                    lse_s[st * kBlockM + lane + 32 * u] = -ri[u].x;
-                    dlt_s[st * kBlockM + lane + 32 * u] = -ri[u].y;
-                }
+            if (lane == 0) {
+                bar.items[slot] = it;
+                mbar_arrive(&bar.item_full[slot]);
             }
             __syncwarp();
-            load_tile<D, ElemBf16>(smem + L::kRing0 + st * L::kTile, &maps.q, &maps.q8, p.q,
-                                   cq + qt * kBlockM, T_q, q_stride, h * D, &bar.ring_full[st], lane);
-            load_tile<D, ElemBf16>(smem + L::kRing1 + st * L::kTile, &maps.dout, &maps.dout8, p.dout,
-                                   cq + qt * kBlockM, T_q, q_stride, h * D, &bar.ring_full[st], lane);
-            ++issued[st];
+            ++item_n;
+            if (idx < 0) break;
+            int qt0, n_qt;
+            item_rows(it, qt0, n_qt);
+            const int n_steps = G * n_qt;
+            if (n_steps == 0) continue;
+            const int cq = p.cu_q[it.b], ck = p.cu_k[it.b];
+            const int L_q = p.cu_q[it.b + 1] - cq;
+            const int hk = it.head, k0 = it.tile * kBlockN;
+            // K and V once the previous item's last products that read them are done
+            if (!(ok = mbar_wait_warp(bar.fixed_empty, (fixed_n & 1) ^ 1, bar.abort_flag, status))) break;
+            load_tile<D, ElemBf16>(smem + L::kFixed0, &maps.k, &maps.k8, p.k, ck + k0, T_k, kv_stride,
+                                   hk * D, bar.fixed_full, lane);
+            load_tile<D, ElemBf16>(smem + L::kFixed1, &maps.v, &maps.v8, p.v, ck + k0, T_k, kv_stride,
+                                   hk * D, bar.fixed_full, lane);
+            ++fixed_n;
+            for (int n = 0; n < n_steps; ++n, ++ring_n) {
+                const int st = ring_n & 1;
+                const int h = hk * G + n / n_qt, qt = qt0 + n % n_qt;
+                if (!(ok = mbar_wait_warp(&bar.ring_empty[st], ((ring_n >> 1) & 1) ^ 1, bar.abort_flag, status)))
+                    break;
+                {
+                    // the tile's 128 rows of {lse * log2(e), Delta}, staged negated (the
+                    // element-wise warps add them): four loads per lane in flight at once
+                    // (rows past the sequence are masked: any finite value)
+                    const float2* src = p.rowinfo + h * p.rows_cap + cq + qt * kBlockM;
+                    float2 ri[kBlockM / 32];
+#pragma unroll
+                    for (int u = 0; u < kBlockM / 32; ++u) {
+                        const int r = lane + 32 * u;
+                        ri[u] = qt * kBlockM + r < L_q ? src[r] : make_float2(0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int u = 0; u < kBlockM / 32; ++u) {
+                        lse_s[st * kBlockM + lane + 32 * u] = -ri[u].x;
+                        dlt_s[st * kBlockM + lane + 32 * u] = -ri[u].y;
+                    }
+                }
+                __syncwarp();
+                load_tile<D, ElemBf16>(smem + L::kRing0 + st * L::kTile, &maps.q, &maps.q8, p.q,
+                                       cq + qt * kBlockM, T_q, q_stride, h * D, &bar.ring_full[st], lane);
+                load_tile<D, ElemBf16>(smem + L::kRing1 + st * L::kTile, &maps.dout, &maps.dout8, p.dout,
+                                       cq + qt * kBlockM, T_q, q_stride, h * D, &bar.ring_full[st], lane);
+                ++issued[st];
+            }
+            if (!ok) break;
         }
         if (!ok && lane == 0) {
             const unsigned long long t0 = global_timer_ns();
-            bwd_drain(bar.fixed_full, 1, t0);
+            bwd_drain(bar.fixed_full, fixed_n, t0);
             bwd_drain(&bar.ring_full[0], issued[0], t0);
             bwd_drain(&bar.ring_full[1], issued[1], t0);
         }
@@ -300,10 +358,8 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
             const uint64_t dq_mn = smem_desc_sw128(smem_u32(smem + L::kRing0), T::kChunkBytes, 1024);
             const uint64_t dd_mn = smem_desc_sw128(smem_u32(smem + L::kRing1), T::kChunkBytes, 1024);
             const uint32_t hi_k = static_cast<uint32_t>(dk_ >> 32), hi_mn = static_cast<uint32_t>(dq_mn >> 32);
-            bool ok = mbar_wait(bar.fixed_full, 0, bar.abort_flag, status);
-            tc_fence_after();
             // S^T = K Q^T for step m (Q of ring stage m & 1, K-major operands, K = D)
-            auto issue_s = [&](int m) {
+            auto issue_s = [&](uint32_t m) {
                 const uint32_t ring = ((m & 1) * L::kTile) >> 4;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -313,53 +369,76 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                 }
                 mma_commit(bar.s_full);
             };
-            // Order per step n: dP^T(n), dV(n) once P^T(n) is stored, S^T(n+1) once
-            // the element-wise warps have loaded P^T(n) (it overwrites those
-            // columns; dV(n), issued before it, reads them first), dK(n) once
-            // dS^T(n) is stored.  The S^T of the next step so runs while dS^T is
-            // formed.  dP^T(n+1) overwrites dS^T(n) and follows dK(n).
-            if (ok && n_steps > 0) {
-                ok = mbar_wait(&bar.ring_full[0], 0, bar.abort_flag, status);
+            uint32_t g = 0, fixed_n = 0, acc_n = 0, item_n = 0;
+            bool ok = true;
+            for (;;) {
+                const int slot = item_n & 1;
+                if (!(ok = mbar_wait(&bar.item_full[slot], (item_n >> 1) & 1, bar.abort_flag, status))) break;
+                const BwdItem it = bar.items[slot];
+                mbar_arrive(&bar.item_empty[slot]);
+                ++item_n;
+                if (it.idx < 0) break;
+                const int n_steps = G * it.a1;
+                if (n_steps == 0) continue;
+                if (!(ok = mbar_wait(bar.fixed_full, fixed_n & 1, bar.abort_flag, status))) break;
+                ++fixed_n;
+                if (!(ok = mbar_wait(&bar.ring_full[g & 1], (g >> 1) & 1, bar.abort_flag, status))) break;
                 tc_fence_after();
-                if (ok) issue_s(0);
-            }
-            for (int n = 0; n < n_steps && ok; ++n) {
-                const int st = n & 1;
-                const uint32_t ring = (st * L::kTile) >> 4;
-                // dP^T = V dout^T (K-major operands, K = D)
+                issue_s(g);
+                // Order per step m: dP^T(m), dV(m) once P^T(m) is stored, S^T(m+1) once
+                // the element-wise warps have loaded P^T(m) (it overwrites those
+                // columns; dV(m), issued before it, reads them first), dK(m) once
+                // dS^T(m) is stored.  The S^T of the next step so runs while dS^T is
+                // formed.  dP^T(m+1) overwrites dS^T(m) and follows dK(m).
+                for (int n = 0; n < n_steps && ok; ++n) {
+                    const uint32_t m = g + n;
+                    const int st = m & 1;
+                    const uint32_t ring = (st * L::kTile) >> 4;
+                    // dP^T = V dout^T (K-major operands, K = D)
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * T::kChunkBytes + (kk & 3) * 32) >> 4;
-                    mma_ss_lh<idesc_ss>(tmem + kDP, static_cast<uint32_t>(dv_) + off, hi_k,
-                                        static_cast<uint32_t>(dd_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(bar.dp_full);
-                // dV += P^T dout (A from tensor memory, B MN-major, K = 128 query rows)
-                if (!(ok = mbar_wait(bar.p_ready, n & 1, bar.abort_flag, status))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kBlockM / 16; ++kk)
-                    mma_ts_lh<idesc_ts>(tmem + kDV, tmem + kS + bwd_kcol(kk),
-                                        static_cast<uint32_t>(dd_mn) + ring + ((kk * 16 * 128) >> 4), hi_mn,
-                                        (n > 0 || kk > 0) ? 1u : 0u);
-                if (n + 1 < n_steps) {
-                    if (!(ok = mbar_wait(&bar.ring_full[(n + 1) & 1], ((n + 1) >> 1) & 1, bar.abort_flag, status)))
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk >> 2) * T::kChunkBytes + (kk & 3) * 32) >> 4;
+                        mma_ss_lh<idesc_ss>(tmem + kDP, static_cast<uint32_t>(dv_) + off, hi_k,
+                                            static_cast<uint32_t>(dd_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar.dp_full);
+                    if (!(ok = mbar_wait(bar.p_ready, m & 1, bar.abort_flag, status))) break;
+                    // the first dV of an item overwrites the accumulators: the previous
+                    // item's must have been read out
+                    if (n == 0 && acc_n > 0 &&
+                        !(ok = mbar_wait(bar.acc_free, (acc_n - 1) & 1, bar.abort_flag, status)))
                         break;
-                    if (!(ok = mbar_wait(bar.p_read, n & 1, bar.abort_flag, status))) break;
                     tc_fence_after();
-                    issue_s(n + 1);
-                }
-                // dK += dS^T Q
-                if (!(ok = mbar_wait(bar.ds_ready, n & 1, bar.abort_flag, status))) break;
-                tc_fence_after();
+                    // dV += P^T dout (A from tensor memory, B MN-major, K = 128 query rows)
 #pragma unroll
-                for (int kk = 0; kk < kBlockM / 16; ++kk)
-                    mma_ts_lh<idesc_ts>(tmem + kDK, tmem + kDP + bwd_kcol(kk),
-                                        static_cast<uint32_t>(dq_mn) + ring + ((kk * 16 * 128) >> 4), hi_mn,
-                                        (n > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(&bar.ring_empty[st]);
+                    for (int kk = 0; kk < kBlockM / 16; ++kk)
+                        mma_ts_lh<idesc_ts>(tmem + kDV, tmem + kS + bwd_kcol(kk),
+                                            static_cast<uint32_t>(dd_mn) + ring + ((kk * 16 * 128) >> 4), hi_mn,
+                                            (n > 0 || kk > 0) ? 1u : 0u);
+                    if (n + 1 < n_steps) {
+                        if (!(ok = mbar_wait(&bar.ring_full[(m + 1) & 1], ((m + 1) >> 1) & 1, bar.abort_flag,
+                                             status)))
+                            break;
+                        if (!(ok = mbar_wait(bar.p_read, m & 1, bar.abort_flag, status))) break;
+                        tc_fence_after();
+                        issue_s(m + 1);
+                    }
+                    // dK += dS^T Q
+                    if (!(ok = mbar_wait(bar.ds_ready, m & 1, bar.abort_flag, status))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kBlockM / 16; ++kk)
+                        mma_ts_lh<idesc_ts>(tmem + kDK, tmem + kDP + bwd_kcol(kk),
+                                            static_cast<uint32_t>(dq_mn) + ring + ((kk * 16 * 128) >> 4), hi_mn,
+                                            (n > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&bar.ring_empty[st]);
+                }
+                if (!ok) break;
+                mma_commit(bar.fixed_empty);  // K and V may be reloaded
+                mma_commit(bar.acc_done);
+                g += n_steps;
+                ++acc_n;
             }
-            mma_commit(bar.acc_done);
         }
         __syncwarp();
     } else {
@@ -367,130 +446,161 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
         const int quarter = warp & 3;                       // TMEM lane quarter
         const int ch = warp >> 2;                           // query columns 64 ch .. 64 ch + 63
         const int jj = quarter * 32 + lane;                 // key row of the tile (TMEM lane)
-        const int j = k0 + jj;                              // key index in the sequence
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-        // query rows that see key j: [i_lo, i_hi] (empty when j is past the keys)
-        int i_lo = 0, i_hi = L_q - 1;
-        if (p.causal || p.window > 0) i_lo = max(0, j - delta_k);
-        if (p.window > 0) i_hi = min(i_hi, j - delta_k + p.window - 1);
-        if (j >= L_k) i_hi = -1;
-        const unsigned i_span = i_hi >= i_lo ? static_cast<unsigned>(i_hi - i_lo) : 0u;
-        const int i_base = i_hi >= i_lo ? i_lo : (1 << 30);
         const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+        uint32_t g = 0, acc_n = 0, item_n = 0;
         bool ok = true;
-        for (int n = 0; n < n_steps; ++n) {
-            const int st = n & 1;
-            const int qt = qt0 + n % n_qt;
-            if (!(ok = mbar_wait_warp(bar.s_full, n & 1, bar.abort_flag, status))) break;
-            // the producer's stores of this step's logsumexp and Delta rows are
-            // released by its arrival on ring_full (already complete: the MMA
-            // warp waited for it before the products this wait observed)
-            if (!(ok = mbar_wait_warp(&bar.ring_full[st], (n >> 1) & 1, bar.abort_flag, status))) break;
-            tc_fence_after();
-            const float* nl2 = lse_s + st * kBlockM;  // -lse * log2(e) per query column
-            const float* ndl = dlt_s + st * kBlockM;  // -Delta per query column
-            // every pair of this warp's keys and query columns visible?  Then the
-            // loops below skip the mask (every tile of a non-causal sequence but
-            // its ragged last one)
-            const int i0 = qt * kBlockM + ch * 64;
-            const bool full = __all_sync(0xffffffffu, i_span != 0u && i_base <= i0 &&
-                                                          i0 + 63 <= i_base + static_cast<int>(i_span));
-            // P^T = exp2(s * log2(e) / sqrt(D) - lse * log2(e)) on visible pairs, as
-            // bf16 at bwd_pcol(c); the second chunk's load is in flight while the
-            // first is computed
-            {
-                uint32_t sbuf[2][32];
-                tmem_ld32(tmem + lane_addr + kS + ch * 64, sbuf[0]);
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int c = 2 * ch + cc;
-                    tmem_wait_ld();
-                    if (cc == 0) tmem_ld32(tmem + lane_addr + kS + ch * 64 + 32, sbuf[1]);
-                    const uint32_t* sr = sbuf[cc];
-                    // scale and shift as packed pairs, then the mask (only on tiles
-                    // where some pair of this warp is not visible)
-                    float pv[32];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        const float4 nl = *reinterpret_cast<const float4*>(nl2 + c * 32 + e);
-                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), scale2,
-                                         f2_pack(nl.x, nl.y)),
-                                  pv[e], pv[e + 1]);
-                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3])), scale2,
-                                         f2_pack(nl.z, nl.w)),
-                                  pv[e + 2], pv[e + 3]);
-                    }
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) pv[e] = ex2_approx(pv[e]);
-                    if (!full) {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int i = qt * kBlockM + c * 32 + e;
-                            pv[e] = static_cast<unsigned>(i - i_base) <= i_span ? pv[e] : 0.f;
-                        }
-                    }
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) pk[e / 2] = pack_bf16x2(pv[e], pv[e + 1]);
-                    tmem_st16(tmem + lane_addr + kS + bwd_pcol(c), pk);
-                }
-            }
-            tmem_wait_st();
-            tc_fence_before();
+        for (;;) {
+            const int slot = item_n & 1;
+            if (!(ok = mbar_wait_warp(&bar.item_full[slot], (item_n >> 1) & 1, bar.abort_flag, status))) break;
+            const BwdItem it = bar.items[slot];
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar.p_ready);
-            // dS^T = P^T (dP^T - Delta) from the stored bf16 P^T, as bf16 at
-            // kDP + bwd_pcol(c)
-            if (!(ok = mbar_wait_warp(bar.dp_full, n & 1, bar.abort_flag, status))) break;
-            tc_fence_after();
-            {
-                uint32_t dbuf[2][32], pbuf[2][16];
-                tmem_ld32(tmem + lane_addr + kDP + ch * 64, dbuf[0]);
-                tmem_ld16(tmem + lane_addr + kS + bwd_pcol(2 * ch), pbuf[0]);
+            if (lane == 0) mbar_arrive(&bar.item_empty[slot]);
+            ++item_n;
+            if (it.idx < 0) break;
+            const int hk = it.head;
+            const int cq = p.cu_q[it.b], ck = p.cu_k[it.b];
+            const int L_q = p.cu_q[it.b + 1] - cq, L_k = p.cu_k[it.b + 1] - ck;
+            const int k0 = it.tile * kBlockN;
+            const int delta_k = L_k - L_q;
+            const int j = k0 + jj;                          // key index in the sequence
+            int qt0, n_qt;
+            item_rows(it, qt0, n_qt);
+            const int n_steps = G * n_qt;
+            if (n_steps == 0) {
+                // no query sees these keys: their gradients are zero (this warp's
+                // half of the columns of its rows)
+                if (j < L_k) {
+                    const long long off = (static_cast<long long>(ck) + j) * kv_pitch + hk * D * 2 + ch * D;
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int c = 2 * ch + cc;
-                    tmem_wait_ld();
-                    if (cc == 0) {
-                        tmem_ld32(tmem + lane_addr + kDP + ch * 64 + 32, dbuf[1]);
-                        tmem_ld16(tmem + lane_addr + kS + bwd_pcol(c + 1), pbuf[1]);
-                    } else {
-                        // every P^T value of this warp is in registers: the next S^T may land
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(bar.p_read);
+                    for (int c = 0; c < D / 16; ++c) {
+                        reinterpret_cast<uint4*>(p.dk + off)[c] = make_uint4(0u, 0u, 0u, 0u);
+                        reinterpret_cast<uint4*>(p.dv + off)[c] = make_uint4(0u, 0u, 0u, 0u);
                     }
-                    const uint32_t* dr = dbuf[cc];
-                    const uint32_t* pr = pbuf[cc];
-                    // dS = P (dP - Delta) on packed pairs; a masked pair has P = 0 and a
-                    // finite dP - Delta (rows past the sequence stage Delta = 0), so it
-                    // stays 0
-                    uint32_t dk16[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        const float4 nd = *reinterpret_cast<const float4*>(ndl + c * 32 + e);
-                        float ds[4];
-#pragma unroll
-                        for (int u = 0; u < 4; u += 2) {
-                            const uint32_t w = pr[(e + u) / 2];
-                            const uint64_t p2 = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-                            const uint64_t d2 = f2_add(f2_pack(__uint_as_float(dr[e + u]), __uint_as_float(dr[e + u + 1])),
-                                                       u == 0 ? f2_pack(nd.x, nd.y) : f2_pack(nd.z, nd.w));
-                            f2_unpack(f2_mul(p2, d2), ds[u], ds[u + 1]);
-                        }
-                        dk16[e / 2] = pack_bf16x2(ds[0], ds[1]);
-                        dk16[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
-                    }
-                    tmem_st16(tmem + lane_addr + kDP + bwd_pcol(c), dk16);
                 }
+                continue;
             }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar.ds_ready);
-        }
-        if (ok) ok = mbar_wait_warp(bar.acc_done, 0, bar.abort_flag, status);
-        if (ok) {
+            // query rows that see key j: [i_lo, i_hi] (empty when j is past the keys)
+            int i_lo = 0, i_hi = L_q - 1;
+            if (p.causal || p.window > 0) i_lo = max(0, j - delta_k);
+            if (p.window > 0) i_hi = min(i_hi, j - delta_k + p.window - 1);
+            if (j >= L_k) i_hi = -1;
+            const unsigned i_span = i_hi >= i_lo ? static_cast<unsigned>(i_hi - i_lo) : 0u;
+            const int i_base = i_hi >= i_lo ? i_lo : (1 << 30);
+            for (int n = 0; n < n_steps; ++n) {
+                const uint32_t m = g + n;  // step count across items
+                const int st = m & 1;
+                const int qt = qt0 + n % n_qt;
+                if (!(ok = mbar_wait_warp(bar.s_full, m & 1, bar.abort_flag, status))) break;
+                // the producer's stores of this step's logsumexp and Delta rows are
+                // released by its arrival on ring_full (already complete: the MMA
+                // warp waited for it before the products this wait observed)
+                if (!(ok = mbar_wait_warp(&bar.ring_full[st], (m >> 1) & 1, bar.abort_flag, status))) break;
+                tc_fence_after();
+                const float* nl2 = lse_s + st * kBlockM;  // -lse * log2(e) per query column
+                const float* ndl = dlt_s + st * kBlockM;  // -Delta per query column
+                // every pair of this warp's keys and query columns visible?  Then the
+                // loops below skip the mask (every tile of a non-causal sequence but
+                // its ragged last one)
+                const int i0 = qt * kBlockM + ch * 64;
+                const bool full = __all_sync(0xffffffffu, i_span != 0u && i_base <= i0 &&
+                                                              i0 + 63 <= i_base + static_cast<int>(i_span));
+                // P^T = exp2(s * log2(e) / sqrt(D) - lse * log2(e)) on visible pairs, as
+                // bf16 at bwd_pcol(c); the second chunk's load is in flight while the
+                // first is computed
+                {
+                    uint32_t sbuf[2][32];
+                    tmem_ld32(tmem + lane_addr + kS + ch * 64, sbuf[0]);
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int c = 2 * ch + cc;
+                        tmem_wait_ld();
+                        if (cc == 0) tmem_ld32(tmem + lane_addr + kS + ch * 64 + 32, sbuf[1]);
+                        const uint32_t* sr = sbuf[cc];
+                        // scale and shift as packed pairs, then the mask (only on tiles
+                        // where some pair of this warp is not visible)
+                        float pv[32];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            const float4 nl = *reinterpret_cast<const float4*>(nl2 + c * 32 + e);
+                            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), scale2,
+                                             f2_pack(nl.x, nl.y)),
+                                      pv[e], pv[e + 1]);
+                            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3])), scale2,
+                                             f2_pack(nl.z, nl.w)),
+                                      pv[e + 2], pv[e + 3]);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) pv[e] = ex2_approx(pv[e]);
+                        if (!full) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) {
+                                const int i = qt * kBlockM + c * 32 + e;
+                                pv[e] = static_cast<unsigned>(i - i_base) <= i_span ? pv[e] : 0.f;
+                            }
+                        }
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) pk[e / 2] = pack_bf16x2(pv[e], pv[e + 1]);
+                        tmem_st16(tmem + lane_addr + kS + bwd_pcol(c), pk);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar.p_ready);
+                // dS^T = P^T (dP^T - Delta) from the stored bf16 P^T, as bf16 at
+                // kDP + bwd_pcol(c)
+                if (!(ok = mbar_wait_warp(bar.dp_full, m & 1, bar.abort_flag, status))) break;
+                tc_fence_after();
+                {
+                    uint32_t dbuf[2][32], pbuf[2][16];
+                    tmem_ld32(tmem + lane_addr + kDP + ch * 64, dbuf[0]);
+                    tmem_ld16(tmem + lane_addr + kS + bwd_pcol(2 * ch), pbuf[0]);
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int c = 2 * ch + cc;
+                        tmem_wait_ld();
+                        if (cc == 0) {
+                            tmem_ld32(tmem + lane_addr + kDP + ch * 64 + 32, dbuf[1]);
+                            tmem_ld16(tmem + lane_addr + kS + bwd_pcol(c + 1), pbuf[1]);
+                        } else {
+                            // every P^T value of this warp is in registers: the next S^T may land
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(bar.p_read);
+                        }
+                        const uint32_t* dr = dbuf[cc];
+                        const uint32_t* pr = pbuf[cc];
+                        // dS = P (dP - Delta) on packed pairs; a masked pair has P = 0 and a
+                        // finite dP - Delta (rows past the sequence stage Delta = 0), so it
+                        // stays 0
+                        uint32_t dk16[16];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            const float4 nd = *reinterpret_cast<const float4*>(ndl + c * 32 + e);
+                            float ds[4];
+#pragma unroll
+                            for (int u = 0; u < 4; u += 2) {
+                                const uint32_t w = pr[(e + u) / 2];
+                                const uint64_t p2 = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+                                const uint64_t d2 = f2_add(f2_pack(__uint_as_float(dr[e + u]), __uint_as_float(dr[e + u + 1])),
+                                                           u == 0 ? f2_pack(nd.x, nd.y) : f2_pack(nd.z, nd.w));
+                                f2_unpack(f2_mul(p2, d2), ds[u], ds[u + 1]);
+                            }
+                            dk16[e / 2] = pack_bf16x2(ds[0], ds[1]);
+                            dk16[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+                        }
+                        tmem_st16(tmem + lane_addr + kDP + bwd_pcol(c), dk16);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar.ds_ready);
+            }
+            if (!ok) break;
+            if (!(ok = mbar_wait_warp(bar.acc_done, acc_n & 1, bar.abort_flag, status))) break;
             tc_fence_after();
             // this warp's half of the D columns of its 32 key rows
             const bool valid = j < L_k;
@@ -499,13 +609,20 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
             uint8_t* base_k = p.dk + (static_cast<long long>(ck) + k0) * kv_pitch + col;
             bwd_store_rows<D / 2>(tmem + lane_addr + kDV + ch * (D / 2), 1.f, base_v, kv_pitch, jj, valid);
             bwd_store_rows<D / 2>(tmem + lane_addr + kDK + ch * (D / 2), p.scale, base_k, kv_pitch, jj, valid);
+            // the accumulators are in registers: the next item's first dV may overwrite them
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar.acc_free);
+            g += n_steps;
+            ++acc_n;
         }
     }
     bwd_teardown<D>(bar, tmem, warp);
 }
 
 // ---------------------------------------------------------------------------
-// dQ: one CTA per (query tile qt, query head h, sequence b) = blockIdx (x, y, z).
+// dQ: items (query tile qt, query head h, sequence b) from the list of query
+// tiles, longest first.
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
@@ -515,55 +632,69 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int hk = h / (p.H / p.H_kv);
-    const int cq = p.cu_q[b], ck = p.cu_k[b];
-    const int L_q = p.cu_q[b + 1] - cq, L_k = p.cu_k[b + 1] - ck;
-    const int q0 = qt * kBlockM;
-    if (q0 >= L_q) return;  // the whole CTA, before any barrier
-    int kt_lo, kt_hi;
-    rows_key_range(q0, kBlockM, L_q, L_k, p.causal != 0, p.window, kt_lo, kt_hi);
-    const int n_steps = kt_hi - kt_lo;
-    const long long q_pitch = static_cast<long long>(p.H) * D * 2;
-    if (n_steps <= 0) {
-        // these rows see no key: dq is zero
-        const int rows = min(L_q - q0, kBlockM);
-        for (int idx = threadIdx.x; idx < rows * (D / 8); idx += blockDim.x) {
-            const int r = idx / (D / 8), c = idx % (D / 8);
-            *reinterpret_cast<uint4*>(p.dq + (static_cast<long long>(cq) + q0 + r) * q_pitch + h * D * 2 +
-                                      c * 16) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        return;
-    }
-
     const BwdBars bar = bwd_setup<D>(smem, warp);
     const uint32_t tmem = *bar.tmem_slot;
     unsigned* status = &g_va_status;
     constexpr uint32_t kS = 0, kDP = 128, kDQ = 256;  // tensor-memory columns
+    const long long q_pitch = static_cast<long long>(p.H) * D * 2;
+    const int n_items = min(max(p.hdr_q->n_tiles, 0), p.cap_q) * p.H;
+    const int G = p.H / p.H_kv;
 
     if (warp == kBwdLoadWarp) {
         // ------------------------------------------------------------ producer
         const int T_q = p.cu_q[p.batch], T_k = p.cu_k[p.batch];
         const int q_stride = p.H * D * 2, kv_stride = p.H_kv * D * 2;
-        uint32_t issued[2] = {0, 0};
+        uint32_t ring_n = 0, fixed_n = 0, item_n = 0, issued[2] = {0, 0};
         bool ok = true;
-        load_tile<D, ElemBf16>(smem + L::kFixed0, &maps.q, &maps.q8, p.q, cq + q0, T_q, q_stride, h * D,
-                               bar.fixed_full, lane);
-        load_tile<D, ElemBf16>(smem + L::kFixed1, &maps.dout, &maps.dout8, p.dout, cq + q0, T_q, q_stride,
-                               h * D, bar.fixed_full, lane);
-        for (int n = 0; n < n_steps; ++n) {
-            const int st = n & 1, kt = kt_lo + n;
-            if (!(ok = mbar_wait_warp(&bar.ring_empty[st], ((n >> 1) & 1) ^ 1, bar.abort_flag, status)))
+        for (;;) {
+            // claim the next item (longest first across the grid) and publish it
+            int idx = -1;
+            if (lane == 0) {
+                const int t = atomicAdd(&p.hdr_q->next_item, 1);
+                idx = t < n_items ? t : -1;
+            }
+            idx = __shfl_sync(0xffffffffu, idx, 0);
+            BwdItem it{idx, 0, 0, 0, 0, 0, {0, 0}};
+            if (idx >= 0) {
+                const TileEntry e = p.list_q[idx / p.H];
+                it = BwdItem{idx, e.b, e.qt, e.kt_lo, e.kt_hi, idx % p.H, {0, 0}};
+            }
+            const int slot = item_n & 1;
+            if (!(ok = mbar_wait_warp(&bar.item_empty[slot], ((item_n >> 1) & 1) ^ 1, bar.abort_flag, status)))
                 break;
-            load_tile<D, ElemBf16>(smem + L::kRing0 + st * L::kTile, &maps.k, &maps.k8, p.k,
-                                   ck + kt * kBlockN, T_k, kv_stride, hk * D, &bar.ring_full[st], lane);
-            load_tile<D, ElemBf16>(smem + L::kRing1 + st * L::kTile, &maps.v, &maps.v8, p.v,
-                                   ck + kt * kBlockN, T_k, kv_stride, hk * D, &bar.ring_full[st], lane);
-            ++issued[st];
+            if (lane == 0) {
+                bar.items[slot] = it;
+                mbar_arrive(&bar.item_full[slot]);
+            }
+            __syncwarp();
+            ++item_n;
+            if (idx < 0) break;
+            const int n_steps = it.a1 - it.a0;
+            if (n_steps <= 0) continue;
+            const int cq = p.cu_q[it.b], ck = p.cu_k[it.b];
+            const int h = it.head, hk = h / G, q0 = it.tile * kBlockM;
+            // Q and dout once the previous item's last products that read them are done
+            if (!(ok = mbar_wait_warp(bar.fixed_empty, (fixed_n & 1) ^ 1, bar.abort_flag, status))) break;
+            load_tile<D, ElemBf16>(smem + L::kFixed0, &maps.q, &maps.q8, p.q, cq + q0, T_q, q_stride, h * D,
+                                   bar.fixed_full, lane);
+            load_tile<D, ElemBf16>(smem + L::kFixed1, &maps.dout, &maps.dout8, p.dout, cq + q0, T_q, q_stride,
+                                   h * D, bar.fixed_full, lane);
+            ++fixed_n;
+            for (int n = 0; n < n_steps; ++n, ++ring_n) {
+                const int st = ring_n & 1, kt = it.a0 + n;
+                if (!(ok = mbar_wait_warp(&bar.ring_empty[st], ((ring_n >> 1) & 1) ^ 1, bar.abort_flag, status)))
+                    break;
+                load_tile<D, ElemBf16>(smem + L::kRing0 + st * L::kTile, &maps.k, &maps.k8, p.k,
+                                       ck + kt * kBlockN, T_k, kv_stride, hk * D, &bar.ring_full[st], lane);
+                load_tile<D, ElemBf16>(smem + L::kRing1 + st * L::kTile, &maps.v, &maps.v8, p.v,
+                                       ck + kt * kBlockN, T_k, kv_stride, hk * D, &bar.ring_full[st], lane);
+                ++issued[st];
+            }
+            if (!ok) break;
         }
         if (!ok && lane == 0) {
             const unsigned long long t0 = global_timer_ns();
-            bwd_drain(bar.fixed_full, 1, t0);
+            bwd_drain(bar.fixed_full, fixed_n, t0);
             bwd_drain(&bar.ring_full[0], issued[0], t0);
             bwd_drain(&bar.ring_full[1], issued[1], t0);
         }
@@ -578,10 +709,8 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
             const uint64_t dv_k = smem_desc_sw128(smem_u32(smem + L::kRing1), 16, 1024);
             const uint64_t dk_mn = smem_desc_sw128(smem_u32(smem + L::kRing0), T::kChunkBytes, 1024);
             const uint32_t hi_k = static_cast<uint32_t>(dq_ >> 32), hi_mn = static_cast<uint32_t>(dk_mn >> 32);
-            bool ok = mbar_wait(bar.fixed_full, 0, bar.abort_flag, status);
-            tc_fence_after();
             // S = Q K^T for step m (K of ring stage m & 1, K-major operands, K = D)
-            auto issue_s = [&](int m) {
+            auto issue_s = [&](uint32_t m) {
                 const uint32_t ring = ((m & 1) * L::kTile) >> 4;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -591,44 +720,67 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                 }
                 mma_commit(bar.s_full);
             };
-            // Order per step n: dP(n), S(n+1) once the element-wise warps have read
-            // S(n), dQ(n) once dS(n) is stored.  The next S so runs while dS is
-            // formed; dP(n+1) overwrites dS(n) and follows dQ(n).
-            if (ok && n_steps > 0) {
-                ok = mbar_wait(&bar.ring_full[0], 0, bar.abort_flag, status);
+            uint32_t g = 0, fixed_n = 0, acc_n = 0, item_n = 0;
+            bool ok = true;
+            for (;;) {
+                const int slot = item_n & 1;
+                if (!(ok = mbar_wait(&bar.item_full[slot], (item_n >> 1) & 1, bar.abort_flag, status))) break;
+                const BwdItem it = bar.items[slot];
+                mbar_arrive(&bar.item_empty[slot]);
+                ++item_n;
+                if (it.idx < 0) break;
+                const int n_steps = it.a1 - it.a0;
+                if (n_steps <= 0) continue;
+                if (!(ok = mbar_wait(bar.fixed_full, fixed_n & 1, bar.abort_flag, status))) break;
+                ++fixed_n;
+                if (!(ok = mbar_wait(&bar.ring_full[g & 1], (g >> 1) & 1, bar.abort_flag, status))) break;
                 tc_fence_after();
-                if (ok) issue_s(0);
-            }
-            for (int n = 0; n < n_steps && ok; ++n) {
-                const int st = n & 1;
-                const uint32_t ring = (st * L::kTile) >> 4;
-                // dP = dout V^T (K-major operands, K = D)
+                issue_s(g);
+                // Order per step m: dP(m), S(m+1) once the element-wise warps have read
+                // S(m), dQ(m) once dS(m) is stored.  The next S so runs while dS is
+                // formed; dP(m+1) overwrites dS(m) and follows dQ(m).
+                for (int n = 0; n < n_steps && ok; ++n) {
+                    const uint32_t m = g + n;
+                    const int st = m & 1;
+                    const uint32_t ring = (st * L::kTile) >> 4;
+                    // dP = dout V^T (K-major operands, K = D)
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * T::kChunkBytes + (kk & 3) * 32) >> 4;
-                    mma_ss_lh<idesc_ss>(tmem + kDP, static_cast<uint32_t>(dd_) + off, hi_k,
-                                        static_cast<uint32_t>(dv_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(bar.dp_full);
-                if (n + 1 < n_steps) {
-                    if (!(ok = mbar_wait(&bar.ring_full[(n + 1) & 1], ((n + 1) >> 1) & 1, bar.abort_flag, status)))
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = ((kk >> 2) * T::kChunkBytes + (kk & 3) * 32) >> 4;
+                        mma_ss_lh<idesc_ss>(tmem + kDP, static_cast<uint32_t>(dd_) + off, hi_k,
+                                            static_cast<uint32_t>(dv_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar.dp_full);
+                    if (n + 1 < n_steps) {
+                        if (!(ok = mbar_wait(&bar.ring_full[(m + 1) & 1], ((m + 1) >> 1) & 1, bar.abort_flag,
+                                             status)))
+                            break;
+                        if (!(ok = mbar_wait(bar.p_read, m & 1, bar.abort_flag, status))) break;
+                        tc_fence_after();
+                        issue_s(m + 1);
+                    }
+                    if (!(ok = mbar_wait(bar.p_ready, m & 1, bar.abort_flag, status))) break;
+                    // the first dQ of an item overwrites the accumulator: the previous
+                    // item's must have been read out
+                    if (n == 0 && acc_n > 0 &&
+                        !(ok = mbar_wait(bar.acc_free, (acc_n - 1) & 1, bar.abort_flag, status)))
                         break;
-                    if (!(ok = mbar_wait(bar.p_read, n & 1, bar.abort_flag, status))) break;
                     tc_fence_after();
-                    issue_s(n + 1);
-                }
-                if (!(ok = mbar_wait(bar.p_ready, n & 1, bar.abort_flag, status))) break;
-                tc_fence_after();
-                // dQ += dS K (A from tensor memory, B = K MN-major, K = 128 keys)
+                    // dQ += dS K (A from tensor memory, B = K MN-major, K = 128 keys)
 #pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    mma_ts_lh<idesc_ts>(tmem + kDQ, tmem + kDP + bwd_kcol(kk),
-                                        static_cast<uint32_t>(dk_mn) + ring + ((kk * 16 * 128) >> 4), hi_mn,
-                                        (n > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                        mma_ts_lh<idesc_ts>(tmem + kDQ, tmem + kDP + bwd_kcol(kk),
+                                            static_cast<uint32_t>(dk_mn) + ring + ((kk * 16 * 128) >> 4), hi_mn,
+                                            (n > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&bar.ring_empty[st]);
                 }
-                mma_commit(&bar.ring_empty[st]);
+                if (!ok) break;
+                mma_commit(bar.fixed_empty);  // Q and dout may be reloaded
+                mma_commit(bar.acc_done);
+                g += n_steps;
+                ++acc_n;
             }
-            mma_commit(bar.acc_done);
         }
         __syncwarp();
     } else {
@@ -636,106 +788,137 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
         const int quarter = warp & 3;        // TMEM lane quarter
         const int ch = warp >> 2;            // key columns 64 ch .. 64 ch + 63
         const int ii = quarter * 32 + lane;  // query row of the tile (TMEM lane)
-        const int i = q0 + ii;
         const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-        const bool row_valid = i < L_q;
-        float l2 = 0.f, dl = 0.f;
-        int lo = 0, hi = -1;
-        if (row_valid) {
-            const size_t row = static_cast<size_t>(cq + i) * p.H + h;
-            const float l = p.lse[row];
-            l2 = l == -INFINITY ? 0.f : l * 1.4426950408889634f;
-            // Delta_i = dout_i . out_i, kept here and stored for the dK/dV kernel
-            const uint4* o4 = reinterpret_cast<const uint4*>(p.out + row * (D * 2));
-            const uint4* g4 = reinterpret_cast<const uint4*>(p.dout + row * (D * 2));
-            float acc = 0.f;
-#pragma unroll 4
-            for (int c = 0; c < D / 8; ++c) {
-                const uint4 a = o4[c], g = g4[c];
-                const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {g.x, g.y, g.z, g.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    acc = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(gv[e] << 16), acc);
-                    acc = fmaf(__uint_as_float(av[e] & 0xFFFF0000u), __uint_as_float(gv[e] & 0xFFFF0000u), acc);
-                }
-            }
-            dl = acc;
-            if (ch == 0) p.rowinfo[h * p.rows_cap + cq + i] = make_float2(l2, acc);
-            row_key_interval(i, L_q, L_k, p.causal != 0, p.window, lo, hi);
-        }
-        const unsigned span = hi >= lo ? static_cast<unsigned>(hi - lo) : 0u;
-        const int base = hi >= lo ? lo : (1 << 30);
-        const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t nl2 = f2_pack(-l2, -l2), ndl2 = f2_pack(-dl, -dl);
+        uint32_t g = 0, acc_n = 0, item_n = 0;
         bool ok = true;
-        for (int n = 0; n < n_steps; ++n) {
-            const int kt = kt_lo + n;
-            if (!(ok = mbar_wait_warp(bar.s_full, n & 1, bar.abort_flag, status))) break;
-            tc_fence_after();
-            // all of this warp's rows see every key of its columns?  (skip the mask)
-            const int k0c = kt * kBlockN + ch * 64;
-            const bool full = __all_sync(0xffffffffu, hi >= lo && lo <= k0c && k0c + 63 <= hi);
-            // P = exp2(s * log2(e) / sqrt(D) - lse * log2(e)) on visible pairs, in
-            // registers; then S may be overwritten by the next step's product
-            float pv[64];
-            {
-                uint32_t sbuf[2][32];
-                tmem_ld32(tmem + lane_addr + kS + ch * 64, sbuf[0]);
-                tmem_ld32(tmem + lane_addr + kS + ch * 64 + 32, sbuf[1]);
-                tmem_wait_ld();
+        for (;;) {
+            const int slot = item_n & 1;
+            if (!(ok = mbar_wait_warp(&bar.item_full[slot], (item_n >> 1) & 1, bar.abort_flag, status))) break;
+            const BwdItem it = bar.items[slot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar.item_empty[slot]);
+            ++item_n;
+            if (it.idx < 0) break;
+            const int h = it.head;
+            const int cq = p.cu_q[it.b], ck = p.cu_k[it.b];
+            const int L_q = p.cu_q[it.b + 1] - cq, L_k = p.cu_k[it.b + 1] - ck;
+            const int q0 = it.tile * kBlockM;
+            const int i = q0 + ii;
+            const bool row_valid = i < L_q;
+            const int n_steps = it.a1 - it.a0;
+            if (n_steps <= 0) {
+                // these rows see no key: dq is zero (this warp's half of the columns)
+                if (row_valid) {
+                    uint4* o = reinterpret_cast<uint4*>(p.dq + (static_cast<long long>(cq) + i) * q_pitch +
+                                                        h * D * 2 + ch * D);
+#pragma unroll
+                    for (int c = 0; c < D / 16; ++c) o[c] = make_uint4(0u, 0u, 0u, 0u);
+                }
+                continue;
+            }
+            float l2 = 0.f, dl = 0.f;
+            int lo = 0, hi = -1;
+            if (row_valid) {
+                const size_t row = static_cast<size_t>(cq + i) * p.H + h;
+                const float l = p.lse[row];
+                l2 = l == -INFINITY ? 0.f : l * 1.4426950408889634f;
+                // Delta_i = dout_i . out_i, kept here and stored for the dK/dV kernel
+                const uint4* o4 = reinterpret_cast<const uint4*>(p.out + row * (D * 2));
+                const uint4* g4 = reinterpret_cast<const uint4*>(p.dout + row * (D * 2));
+                float acc = 0.f;
+#pragma unroll 4
+                for (int c = 0; c < D / 8; ++c) {
+                    const uint4 a = o4[c], gg = g4[c];
+                    const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {gg.x, gg.y, gg.z, gg.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        acc = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(gv[e] << 16), acc);
+                        acc = fmaf(__uint_as_float(av[e] & 0xFFFF0000u), __uint_as_float(gv[e] & 0xFFFF0000u), acc);
+                    }
+                }
+                dl = acc;
+                if (ch == 0) p.rowinfo[h * p.rows_cap + cq + i] = make_float2(l2, acc);
+                row_key_interval(i, L_q, L_k, p.causal != 0, p.window, lo, hi);
+            }
+            const unsigned span = hi >= lo ? static_cast<unsigned>(hi - lo) : 0u;
+            const int base = hi >= lo ? lo : (1 << 30);
+            const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+            const uint64_t nl2 = f2_pack(-l2, -l2), ndl2 = f2_pack(-dl, -dl);
+            for (int n = 0; n < n_steps; ++n) {
+                const int kt = it.a0 + n;
+                const uint32_t m = g + n;  // step count across items
+                if (!(ok = mbar_wait_warp(bar.s_full, m & 1, bar.abort_flag, status))) break;
+                tc_fence_after();
+                // all of this warp's rows see every key of its columns?  (skip the mask)
+                const int k0c = kt * kBlockN + ch * 64;
+                const bool full = __all_sync(0xffffffffu, hi >= lo && lo <= k0c && k0c + 63 <= hi);
+                // P = exp2(s * log2(e) / sqrt(D) - lse * log2(e)) on visible pairs, in
+                // registers; then S may be overwritten by the next step's product
+                float pv[64];
+                {
+                    uint32_t sbuf[2][32];
+                    tmem_ld32(tmem + lane_addr + kS + ch * 64, sbuf[0]);
+                    tmem_ld32(tmem + lane_addr + kS + ch * 64 + 32, sbuf[1]);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar.p_read);
+#pragma unroll
+                    for (int e = 0; e < 64; e += 2)
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(sbuf[e >> 5][e & 31]),
+                                                 __uint_as_float(sbuf[e >> 5][(e & 31) + 1])),
+                                         scale2, nl2),
+                                  pv[e], pv[e + 1]);
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) pv[e] = ex2_approx(pv[e]);
+                    if (!full) {
+#pragma unroll
+                        for (int e = 0; e < 64; ++e)
+                            pv[e] = static_cast<unsigned>(k0c + e - base) <= span ? pv[e] : 0.f;
+                    }
+                }
+                // dS = P (dP - Delta) as bf16 at kDP + bwd_pcol(c), over dP columns read
+                if (!(ok = mbar_wait_warp(bar.dp_full, m & 1, bar.abort_flag, status))) break;
+                tc_fence_after();
+                {
+                    uint32_t dbuf[2][32];
+                    tmem_ld32(tmem + lane_addr + kDP + ch * 64, dbuf[0]);
+                    tmem_ld32(tmem + lane_addr + kDP + ch * 64 + 32, dbuf[1]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        uint32_t dk16[16];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            // a masked pair has P = 0 and a finite dP - Delta: it stays 0
+                            float d0, d1;
+                            f2_unpack(f2_mul(f2_pack(pv[cc * 32 + e], pv[cc * 32 + e + 1]),
+                                             f2_add(f2_pack(__uint_as_float(dbuf[cc][e]), __uint_as_float(dbuf[cc][e + 1])),
+                                                    ndl2)),
+                                      d0, d1);
+                            dk16[e / 2] = pack_bf16x2(d0, d1);
+                        }
+                        tmem_st16(tmem + lane_addr + kDP + bwd_pcol(2 * ch + cc), dk16);
+                    }
+                }
+                tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar.p_read);
-#pragma unroll
-                for (int e = 0; e < 64; e += 2)
-                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sbuf[e >> 5][e & 31]),
-                                             __uint_as_float(sbuf[e >> 5][(e & 31) + 1])),
-                                     scale2, nl2),
-                              pv[e], pv[e + 1]);
-#pragma unroll
-                for (int e = 0; e < 64; ++e) pv[e] = ex2_approx(pv[e]);
-                if (!full) {
-#pragma unroll
-                    for (int e = 0; e < 64; ++e)
-                        pv[e] = static_cast<unsigned>(k0c + e - base) <= span ? pv[e] : 0.f;
-                }
+                if (lane == 0) mbar_arrive(bar.p_ready);
             }
-            // dS = P (dP - Delta) as bf16 at kDP + bwd_pcol(c), over dP columns read
-            if (!(ok = mbar_wait_warp(bar.dp_full, n & 1, bar.abort_flag, status))) break;
-            tc_fence_after();
-            {
-                uint32_t dbuf[2][32];
-                tmem_ld32(tmem + lane_addr + kDP + ch * 64, dbuf[0]);
-                tmem_ld32(tmem + lane_addr + kDP + ch * 64 + 32, dbuf[1]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    uint32_t dk16[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        // a masked pair has P = 0 and a finite dP - Delta: it stays 0
-                        float d0, d1;
-                        f2_unpack(f2_mul(f2_pack(pv[cc * 32 + e], pv[cc * 32 + e + 1]),
-                                         f2_add(f2_pack(__uint_as_float(dbuf[cc][e]), __uint_as_float(dbuf[cc][e + 1])),
-                                                ndl2)),
-                                  d0, d1);
-                        dk16[e / 2] = pack_bf16x2(d0, d1);
-                    }
-                    tmem_st16(tmem + lane_addr + kDP + bwd_pcol(2 * ch + cc), dk16);
-                }
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar.p_ready);
-        }
-        if (ok) ok = mbar_wait_warp(bar.acc_done, 0, bar.abort_flag, status);
-        if (ok) {
+            if (!ok) break;
+            if (!(ok = mbar_wait_warp(bar.acc_done, acc_n & 1, bar.abort_flag, status))) break;
             tc_fence_after();
             // this warp's half of the D columns of its 32 query rows
             uint8_t* base_q = p.dq + (static_cast<long long>(cq) + q0) * q_pitch + h * D * 2 + ch * D;
             bwd_store_rows<D / 2>(tmem + lane_addr + kDQ + ch * (D / 2), p.scale, base_q, q_pitch, ii,
                                   row_valid);
+            // the accumulator is in registers: the next item's first dQ may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar.acc_free);
+            g += n_steps;
+            ++acc_n;
         }
     }
     bwd_teardown<D>(bar, tmem, warp);

@@ -53,6 +53,21 @@ __host__ __device__ __forceinline__ int seq_key_count(const int* cu_k, const int
     return used < cap ? used : cap;
 }
 
+// Query rows of a sequence that see some key of key tile kt (keys [k0,
+// k_last]): [r0, r1] under bottom-right causal alignment and a window of W
+// keys ending at the diagonal (empty when r1 < r0).
+__host__ __device__ __forceinline__ void key_tile_rows(int kt, int L_q, int L_k, bool causal, int window,
+                                                       int& r0, int& r1) {
+    const int k0 = kt * kBlockN;
+    const int k_last = (L_k < k0 + kBlockN ? L_k : k0 + kBlockN) - 1;
+    const int delta_k = L_k - L_q;
+    r0 = 0;
+    r1 = L_q - 1;
+    if (causal || window > 0) r0 = (k0 - delta_k > 0 ? k0 - delta_k : 0);
+    if (window > 0) r1 = (r1 < k_last - delta_k + window - 1 ? r1 : k_last - delta_k + window - 1);
+    if (L_q <= 0 || k0 >= L_k) r1 = r0 - 1;
+}
+
 // Key-tile range of query rows [first, first + rows) clipped to L_q.  The
 // intervals of consecutive rows have non-decreasing ends and overlap or
 // touch, so the union over the rows is the interval of the first non-empty

@@ -124,6 +124,9 @@ int device_setup(int& dev, DeviceInfo*& info) {
     VA_CUDA(cudaFuncSetAttribute(va::build_schedule_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  va::kSortCapacity * 8));
+    VA_CUDA(cudaFuncSetAttribute(va::build_bwd_list_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 va::kSortCapacity * 8));
     VA_CUDA(cudaFuncSetAttribute(va::bwd_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  va::BwdSmem<64>::kAlloc));
     VA_CUDA(cudaFuncSetAttribute(va::bwd_dkdv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -499,8 +502,12 @@ int run_backward(const BwdArgs& g, cudaStream_t stream) {
         }
     }
     if (a.batch == 0) return VA_OK;
-    if (a.batch > 65535 || a.H > 65535)
-        return fail(VA_ERR_UNSUPPORTED, "batch and num_heads must be <= 65535 for the backward grid");
+    // the work lists: one entry per 128-row query tile (dQ) and per 128-key tile (dK/dV)
+    const long long cap_q_ll = static_cast<long long>(a.batch) * ((a.max_q + va::kBlockM - 1) / va::kBlockM);
+    const long long cap_k_ll = static_cast<long long>(a.batch) * ((a.max_k + va::kBlockN - 1) / va::kBlockN);
+    if (cap_q_ll * a.H >= INT_MAX || cap_k_ll * a.H_kv >= INT_MAX)
+        return fail(VA_ERR_UNSUPPORTED, "too many tiles x heads for the backward work lists");
+    const int cap_q = static_cast<int>(cap_q_ll), cap_k = static_cast<int>(cap_k_ll);
     int dev;
     DeviceInfo* info;
     if ((rc = device_setup(dev, info)) != VA_OK) return rc;
@@ -518,9 +525,32 @@ int run_backward(const BwdArgs& g, cudaStream_t stream) {
         (rc = make_tile_map(&maps.k8, a.k, cols_k, rows_k, 8)) != VA_OK ||
         (rc = make_tile_map(&maps.v8, a.v, cols_k, rows_k, 8)) != VA_OK)
         return rc;
-    float2* rowinfo = nullptr;
-    VA_CUDA(ws_alloc(reinterpret_cast<void**>(&rowinfo), static_cast<size_t>(rows_q) * a.H * sizeof(float2),
-                     stream));
+    // workspace: {lse * log2(e), Delta} per (head, query row), two list headers,
+    // the two lists (each with its sort's second buffer)
+    auto up256 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    const size_t ri_bytes = up256(static_cast<size_t>(rows_q) * a.H * sizeof(float2));
+    const size_t lq_bytes = static_cast<size_t>(cap_q) * sizeof(va::TileEntry);
+    const size_t lk_bytes = static_cast<size_t>(cap_k) * sizeof(va::TileEntry);
+    char* ws = nullptr;
+    VA_CUDA(ws_alloc(reinterpret_cast<void**>(&ws), ri_bytes + 512 + up256(2 * lq_bytes) + 2 * lk_bytes, stream));
+    float2* rowinfo = reinterpret_cast<float2*>(ws);
+    auto* hdr_q = reinterpret_cast<va::SchedHeader*>(ws + ri_bytes);
+    auto* hdr_k = reinterpret_cast<va::SchedHeader*>(ws + ri_bytes + 256);
+    auto* scratch_q = reinterpret_cast<va::TileEntry*>(ws + ri_bytes + 512);
+    auto* list_q = scratch_q + cap_q;
+    auto* scratch_k = reinterpret_cast<va::TileEntry*>(ws + ri_bytes + 512 + up256(2 * lq_bytes));
+    auto* list_k = scratch_k + cap_k;
+    auto slots = [](int cap) {
+        int s = 1;
+        while (s < cap && s < va::kSortCapacity) s <<= 1;
+        return s;
+    };
+    if (cap_q > 0)
+        va::build_bwd_list_kernel<<<1, va::kBuildThreads, slots(cap_q) * 8, stream>>>(
+            a.cu_q, a.cu_k, a.batch, a.causal, a.window, 0, cap_q, slots(cap_q), scratch_q, list_q, hdr_q);
+    if (cap_k > 0)
+        va::build_bwd_list_kernel<<<1, va::kBuildThreads, slots(cap_k) * 8, stream>>>(
+            a.cu_q, a.cu_k, a.batch, a.causal, a.window, 1, cap_k, slots(cap_k), scratch_k, list_k, hdr_k);
     va::BwdParams p;
     p.cu_q = a.cu_q;
     p.cu_k = a.cu_k;
@@ -542,21 +572,29 @@ int run_backward(const BwdArgs& g, cudaStream_t stream) {
     p.dv = static_cast<uint8_t*>(g.dv);
     p.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(a.D)));
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)));
-    const dim3 grid_kv(static_cast<unsigned>((std::max(a.max_k, 1) + va::kBlockN - 1) / va::kBlockN),
-                       static_cast<unsigned>(a.H_kv), static_cast<unsigned>(a.batch));
-    const dim3 grid_q(static_cast<unsigned>((std::max(a.max_q, 1) + va::kBlockM - 1) / va::kBlockM),
-                      static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch));
+    p.list_q = list_q;
+    p.hdr_q = hdr_q;
+    p.cap_q = cap_q;
+    p.list_k = list_k;
+    p.hdr_k = hdr_k;
+    p.cap_k = cap_k;
+    // persistent grids, one CTA per SM (fewer when there are fewer items);
     // dQ first: it forms Delta for every query row that sees a key, which the
     // dK/dV kernel reads
+    const int grid_q = static_cast<int>(std::min<long long>(info->num_sms, cap_q_ll * a.H));
+    const int grid_kv = static_cast<int>(std::min<long long>(info->num_sms, cap_k_ll * a.H_kv));
     if (a.D == 64) {
-        va::bwd_dq_kernel<64><<<grid_q, va::kBwdThreads, va::BwdSmem<64>::kAlloc, stream>>>(maps, p);
-        va::bwd_dkdv_kernel<64><<<grid_kv, va::kBwdThreads, va::BwdSmem<64>::kAlloc, stream>>>(maps, p);
+        if (grid_q > 0) va::bwd_dq_kernel<64><<<grid_q, va::kBwdThreads, va::BwdSmem<64>::kAlloc, stream>>>(maps, p);
+        if (grid_kv > 0)
+            va::bwd_dkdv_kernel<64><<<grid_kv, va::kBwdThreads, va::BwdSmem<64>::kAlloc, stream>>>(maps, p);
     } else {
-        va::bwd_dq_kernel<128><<<grid_q, va::kBwdThreads, va::BwdSmem<128>::kAlloc, stream>>>(maps, p);
-        va::bwd_dkdv_kernel<128><<<grid_kv, va::kBwdThreads, va::BwdSmem<128>::kAlloc, stream>>>(maps, p);
+        if (grid_q > 0)
+            va::bwd_dq_kernel<128><<<grid_q, va::kBwdThreads, va::BwdSmem<128>::kAlloc, stream>>>(maps, p);
+        if (grid_kv > 0)
+            va::bwd_dkdv_kernel<128><<<grid_kv, va::kBwdThreads, va::BwdSmem<128>::kAlloc, stream>>>(maps, p);
     }
     cudaError_t le = cudaGetLastError();
-    cudaFreeAsync(rowinfo, stream);
+    cudaFreeAsync(ws, stream);
     if (le != cudaSuccess) return cuda_fail(le, "backward launch");
     return VA_OK;
 }
