@@ -81,6 +81,7 @@ struct PrefillParams {
     float* lse;
     float scale_log2;  // log2(e) / sqrt(D), times q_scale * k_scale for E4M3 inputs
     float out_mul;     // 1 for bf16; v_scale / o_scale for E4M3 (dequantize V, quantize O)
+    int after_residual;  // the residual variant was launched between the build and this grid
 };
 
 template <int D, class E>
@@ -124,13 +125,16 @@ struct Item {
 static_assert(sizeof(Item) <= 64, "an item must fit its 64-byte ring slot");
 
 __device__ __forceinline__ void decode_item(const PrefillParams& p, int idx, int group, Item& it) {
-    const TileEntry te = p.tiles[idx / p.H];
+    // through L2: the main variant reads the list without a grid-dependency
+    // wait on the grid that wrote it (see the kernel's start)
+    const int4 te = __ldcg(reinterpret_cast<const int4*>(p.tiles) + idx / p.H);
+    static_assert(sizeof(TileEntry) == sizeof(int4), "a list entry is one 16-byte load");
     it.h = idx % p.H;
     it.hk = it.h / group;
-    it.b = te.b;
-    it.qb = te.qt;
-    it.lo = te.kt_lo;
-    it.hi = te.kt_hi;
+    it.b = te.x;
+    it.qb = te.y;
+    it.lo = te.z;
+    it.hi = te.w;
     const int cq = p.cu_q[it.b], ck = p.cu_k[it.b];
     it.L_q = p.cu_q[it.b + 1] - cq;
     it.L_k = seq_key_count(p.cu_k, p.seqused_k, it.b);
@@ -245,8 +249,10 @@ __device__ __forceinline__ void store_row_zero(const PrefillParams& p, size_t ou
 // kRes (bf16 only): the variant that serves the list's second part, the query
 // blocks holding a row that sees few keys, with every role's per-item code
 // also multiplying V by P's bf16 rounding residual (see kResidualMaxKeys); the
-// main variant carries none of that code.  The host launches the main variant,
-// then the residual variant as its programmatic dependent.
+// main variant carries none of that code.  The host launches the residual
+// variant right after the schedule build and the main variant as its
+// programmatic dependent, so the short few-key items run beside the main
+// part's longest ones instead of after its tail.
 template <int D, class E, bool kRes>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
 prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams p) {
@@ -276,6 +282,18 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
     Item* item_slot = reinterpret_cast<Item*>(smem + L::kItems);                   // [2]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if constexpr (kRes) {
+        // Wait for the schedule build, then let the main variant launch.  The
+        // grid is one CTA per SM and the CTAs claim items from one counter, so
+        // the first n_items CTAs serve every item between them; the others
+        // leave before any set-up and hand their SM to the main variant at once.
+        grid_dependency_wait();
+        grid_launch_dependents();
+        const int n_list = min(max(__ldcg(&p.hdr->n_tiles), 0), p.tile_capacity);
+        const int n_main = min(max(__ldcg(&p.hdr->n_main), 0), n_list);
+        if (static_cast<long long>(blockIdx.x) >= static_cast<long long>(n_list - n_main) * p.H) return;
+    }
 
     if (threadIdx.x == 0) {
         for (int x = 0; x < 2; ++x) {
@@ -307,18 +325,16 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
         prefetch_tensormap(&maps.v);
     }
     if constexpr (!kRes) {
-        // The set-up above overlaps the schedule build (programmatic dependent
-        // launch); everything below reads the list it writes.  Once every CTA
-        // is past this wait the list is complete, and the residual variant,
-        // launched next, may start on the SMs this grid leaves as its work runs
-        // out (the list's second part is short).
-        grid_dependency_wait();
-        grid_launch_dependents();
+        // Straight after the schedule build (E4M3) the set-up above overlaps
+        // the build and this wait covers everything below, which reads the
+        // list it writes.  After the residual variant there is no wait here:
+        // this grid launches only once every CTA of that variant is past its
+        // own wait for the completed build, so the list is final and is read
+        // through L2 (the header below, the entries in decode_item); the wait
+        // for the residual variant's completion comes at the exit instead,
+        // which keeps the stream's order for whatever follows.
+        if (!p.after_residual) grid_dependency_wait();
     }
-    // (The residual variant is launched only once every CTA of the main
-    // variant is past its wait for the schedule build, so the list is complete
-    // when it reads it; it waits for the main variant's completion before it
-    // exits, which keeps the stream's order for whatever follows.)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -326,8 +342,8 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
 
     // this variant's part of the list as item indices (block index x H +
     // head): the main part [0, n_main H), the few-key part [n_main H, n_list H)
-    const int n_list = min(max(p.hdr->n_tiles, 0), p.tile_capacity);
-    const int n_main = min(max(p.hdr->n_main, 0), n_list);
+    const int n_list = min(max(__ldcg(&p.hdr->n_tiles), 0), p.tile_capacity);
+    const int n_main = min(max(__ldcg(&p.hdr->n_main), 0), n_list);
     const int item0 = kRes ? n_main * p.H : 0;
     const int n_items = (kRes ? n_list - n_main : n_main) * p.H;
     int* counter = kRes ? &p.hdr->next_item_res : &p.hdr->next_item;
@@ -820,7 +836,7 @@ prefill_fwd_kernel(const __grid_constant__ PrefillMaps maps, const PrefillParams
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    if constexpr (kRes) grid_dependency_wait();
+    if constexpr (!kRes) grid_dependency_wait();
 }
 
 }  // namespace va

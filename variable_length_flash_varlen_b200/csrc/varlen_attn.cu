@@ -300,13 +300,15 @@ va::PrefillParams prefill_params(const Args& a) {
     p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.D)) * qk);
     // E4M3 output code = O / o_scale (o_scale is the output's dequantization scale)
     p.out_mul = a.fp8 ? static_cast<float>(static_cast<double>(a.v_scale) / a.o_scale) : 1.f;
+    p.after_residual = 0;
     return p;
 }
 
-// The prefill kernel follows the schedule build on the same stream as a
-// programmatic dependent launch: its CTAs may start (barriers, tensor memory,
-// tensor-map prefetch) while the build still runs, and wait for the build's
-// completion before reading the list.
+// The prefill kernels follow the schedule build on the same stream as
+// programmatic dependent launches: the first one's CTAs may start while the
+// build still runs and wait for the build's completion before reading the list;
+// the bf16 main variant, launched after the residual variant, starts on the SMs
+// that variant leaves and waits for its completion only at its own exit.
 cudaError_t launch_prefill(const Args& a, const va::PrefillMaps& maps, const va::PrefillParams& p,
                            int grid, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
@@ -322,20 +324,22 @@ cudaError_t launch_prefill(const Args& a, const va::PrefillMaps& maps, const va:
         cfg.dynamicSmemBytes = va::PrefillSmem<128, va::ElemE4m3>::kAlloc;
         return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<128, va::ElemE4m3, false>, maps, p);
     }
-    // bf16: the main variant over the list's main part, then the residual
-    // variant over its few-key part, a programmatic dependent launch of the
-    // main one that starts on the SMs the main one leaves as its work runs out
+    // bf16: the residual variant over the list's few-key part first (its CTAs
+    // without an item leave at once), then the main variant over the main
+    // part as its programmatic dependent, on the SMs the residual one leaves
+    va::PrefillParams pm = p;
+    pm.after_residual = 1;
     cudaError_t e;
     if (a.D == 64) {
         cfg.dynamicSmemBytes = va::PrefillSmem<64, va::ElemBf16>::kAlloc;
-        e = cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<64, va::ElemBf16, false>, maps, p);
+        e = cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<64, va::ElemBf16, true>, maps, p);
         if (e != cudaSuccess) return e;
-        return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<64, va::ElemBf16, true>, maps, p);
+        return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<64, va::ElemBf16, false>, maps, pm);
     }
     cfg.dynamicSmemBytes = va::PrefillSmem<128, va::ElemBf16>::kAlloc;
-    e = cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<128, va::ElemBf16, false>, maps, p);
+    e = cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<128, va::ElemBf16, true>, maps, p);
     if (e != cudaSuccess) return e;
-    return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<128, va::ElemBf16, true>, maps, p);
+    return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<128, va::ElemBf16, false>, maps, pm);
 }
 
 int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
