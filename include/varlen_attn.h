@@ -179,11 +179,14 @@ int varlen_attention_fwd_ex(const void* q, const void* k, const void* v,
  * Copies inputs to the device, runs varlen_attention_fwd on `stream`, copies
  * out and lse back and synchronises `stream` before returning.  Device
  * buffers are allocated and freed stream-ordered inside the call.  Once the
- * inputs reach 8 MiB the batch is split into up to four chunks of whole
- * sequences (balanced by query tokens) and pipelined: each chunk's kernels
- * run on `stream` while the next chunk is copied in and the previous one
- * copied out on two library-owned copy streams (created on the first such
- * call per device); the results are bit-identical to one launch over the
+ * inputs reach 8 MiB the batch is cut, in packed query order, into chunks of
+ * about 1/16 of the query rows (at least 4096): groups of whole sequences,
+ * and pieces of a longer sequence (whole 256-row query blocks with the keys
+ * they can see, so a causal or windowed piece needs only the keys up to its
+ * last row), pipelined: each chunk's kernels run on `stream` while the next
+ * chunk's query rows and new key rows are copied in and the previous chunk's
+ * results copied out on two library-owned copy streams (created on the first
+ * such call per device); the results are bit-identical to one launch over the
  * whole batch.  Because both cu_seqlens arrays are in host memory here, the
  * call checks them before any device work (the checks of
  * varlen_attention_validate_cu_seqlens: cu[0] == 0, never decreasing, no
@@ -236,6 +239,24 @@ int varlen_attention_fwd_noalloc(const void* q, const void* k, const void* v,
 int varlen_attention_schedule(const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
                               int batch, int max_seqlen_q, int causal, int window,
                               int32_t* tiles, int32_t* n_tiles, int capacity, void* stream);
+
+/*
+ * Test-only export: the pipeline plan varlen_attention_fwd_host follows for
+ * these host cu_seqlens arrays (host computation only, no device work).
+ * input_bytes is the size of q, k and v together (the plan is one chunk below
+ * 8 MiB).  Chunk c occupies chunks[9 c .. 9 c + 8] (int64): piece (1 = whole
+ * 256-row query blocks of one sequence, 0 = whole sequences), b0, b1 (the
+ * sequences [b0, b1)), q0, q1 (packed query rows), k_base (packed key row of
+ * the chunk's key 0), k_len (a piece's key count, 0 for whole sequences),
+ * kc0, kc1 (the packed key rows this chunk copies in).  Stores the number of
+ * chunks in *n_chunks and writes them if capacity is at least that number.
+ * Returns VA_ERR_INVALID_ARG for a NULL pointer, batch < 0, window < 0,
+ * cu_seqlens that do not start at 0 or decrease, or a capacity below the
+ * number of chunks (*n_chunks is still set).
+ */
+int varlen_attention_host_chunks(const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                 int batch, int causal, int window, long long input_bytes,
+                                 long long* chunks, int capacity, int* n_chunks);
 
 /*
  * Synchronise the current device, then store the device status word

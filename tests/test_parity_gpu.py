@@ -162,6 +162,40 @@ def test_host_buffer_entry_pipelined_chunks_match_device_entry():
     assert torch.equal(out_h, out_d.cpu()) and torch.equal(lse_h, lse_d.cpu())
 
 
+# Sequences longer than a pipelined chunk are cut into pieces of whole 256-row
+# query blocks, each launched with only the keys its rows can see (below a
+# window, rounded down to a 128-key tile; up to the last row's diagonal when
+# causal or windowed): the same blocks, key tiles and masks as one launch, so
+# bit-identical.  Shapes cover causal with fewer and with more queries than
+# keys, a window with and without causal, and a non-causal piece (every key).
+PIECE_CASES = {
+    "sliding_window_quarter": lambda: workloads.named("sliding_window", scale=0.25),
+    "noncausal_long": lambda: workloads.custom([10000, 500], [10000, 500], 8, 8, 128, False, 0, seed=21),
+    "causal_fewer_queries": lambda: workloads.custom([9000, 100], [12000, 300], 8, 4, 128, True, 0, seed=22),
+    "causal_more_queries": lambda: workloads.custom([9000], [6000], 8, 8, 128, True, 0, seed=23),
+    "window_noncausal": lambda: workloads.custom([20000], [20000], 8, 8, 128, False, 1000, seed=24),
+    "window_fewer_queries": lambda: workloads.custom([9000], [15000], 8, 2, 64, True, 777, seed=25),
+    "gqa_causal": lambda: workloads.named("gqa_causal"),
+}
+
+
+@pytest.mark.parametrize("case", sorted(PIECE_CASES))
+def test_host_buffer_entry_pieces_match_device_entry(case):
+    wl = PIECE_CASES[case]()
+    assert max(wl.lengths_q) > 4096  # at least one sequence is cut into pieces
+    q, k, v = workloads.make_qkv(wl)
+    out_d, lse_d = run_gpu(wl, q, k, v)
+    out_h = torch.full_like(q, float("nan")).pin_memory()
+    lse_h = torch.full((wl.total_q, wl.H), float("nan"), dtype=torch.float32).pin_memory()
+    cq = torch.tensor(wl.cu_q, dtype=torch.int32)
+    ck = torch.tensor(wl.cu_k, dtype=torch.int32)
+    binding.varlen_attention_fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), cq, ck,
+                                      wl.batch, wl.H, wl.H_kv, wl.max_seqlen_q, wl.max_seqlen_k,
+                                      wl.D, wl.causal, wl.window, out_h, lse_h)
+    assert torch.equal(out_h, out_d.cpu()), f"{case}: outputs differ"
+    assert torch.equal(lse_h, lse_d.cpu()), f"{case}: logsumexp differs"
+
+
 # --- decode path -------------------------------------------------------------------
 
 @pytest.mark.parametrize("split_keys", [32, 100, 448, 1024, 5000])

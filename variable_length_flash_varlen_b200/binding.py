@@ -9,7 +9,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from typing import Optional, Tuple
+from typing import List, Optional, Tuple
 
 import torch
 
@@ -34,6 +34,7 @@ SIGNATURES = {
     "varlen_attention_fwd_host": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_fwd_noalloc": (_I, [_P, _P, _P, _P, _P] + [_I] * 8 + [_P, _P, _P]),
     "varlen_attention_schedule": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P]),
+    "varlen_attention_host_chunks": (_I, [_P, _P, _I, _I, _I, ctypes.c_longlong, _P, _I, _P]),
     "varlen_attention_device_status": (_I, [ctypes.POINTER(ctypes.c_uint), _I]),
     "varlen_attention_sync_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint), _I]),
     "varlen_attention_validate_cu_seqlens": (_I, [_P, _I, _I, _I, _I, _P]),
@@ -301,6 +302,25 @@ def validate_cu_seqlens(cu_seqlens: torch.Tensor, batch: int, max_seqlen: int, t
     _check(load().varlen_attention_validate_cu_seqlens(
         cu_seqlens.data_ptr(), batch, max_seqlen, total, int(on_device),
         _stream_ptr(stream) if on_device else None))
+
+
+HOST_CHUNK_FIELDS = ("piece", "b0", "b1", "q0", "q1", "k_base", "k_len", "kc0", "kc1")
+
+
+def host_chunks(cu_seqlens_q, cu_seqlens_k, batch: int, causal: bool, window: int,
+                input_bytes: int) -> List[dict]:
+    """The copy/compute plan varlen_attention_fwd_host follows for these host
+    cu_seqlens (no device work): one dict of HOST_CHUNK_FIELDS per chunk."""
+    cq = torch.as_tensor(cu_seqlens_q, dtype=torch.int32).contiguous()
+    ck = torch.as_tensor(cu_seqlens_k, dtype=torch.int32).contiguous()
+    lib = load()
+    n = ctypes.c_int(0)
+    lib.varlen_attention_host_chunks(cq.data_ptr(), ck.data_ptr(), batch, int(causal), window,
+                                     input_bytes, None, 0, ctypes.byref(n))
+    buf = (ctypes.c_longlong * (9 * max(1, n.value)))()
+    _check(lib.varlen_attention_host_chunks(cq.data_ptr(), ck.data_ptr(), batch, int(causal), window,
+                                            input_bytes, buf, n.value, ctypes.byref(n)))
+    return [dict(zip(HOST_CHUNK_FIELDS, buf[9 * c: 9 * c + 9])) for c in range(n.value)]
 
 
 def device_status(clear: bool = True) -> int:

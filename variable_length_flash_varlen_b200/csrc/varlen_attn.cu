@@ -63,8 +63,10 @@ int cuda_fail(cudaError_t e, const char* what) {
 constexpr int kMaxDevices = 64;
 // Host-buffer entry point: up to this many pipelined chunks, once the inputs
 // reach this size.
-constexpr int kHostChunks = 4;
+constexpr int kHostChunks = 16;
 constexpr size_t kHostChunkMinBytes = size_t(8) << 20;
+// ... and no chunk below this many query rows (each chunk is its own launch)
+constexpr long long kHostChunkMinRows = 4096;
 
 // Shared-memory limits of every prefill kernel variant.
 int set_prefill_attributes() {
@@ -708,6 +710,73 @@ int run_prefill_noalloc(const Args& a, cudaStream_t stream) {
     return VA_OK;
 }
 
+// One chunk of the host-buffer entry point's pipeline: the packed query rows
+// [q0, q1) and, for its kernels, the keys from packed row k_base on.
+struct HostChunk {
+    bool piece;           // part of one sequence (b0) rather than whole sequences [b0, b1)
+    int b0, b1;
+    long long q0, q1;     // packed query rows
+    long long k_base;     // packed key row of the chunk's key 0
+    long long k_len;      // a piece's key count (a group's come from cu_seqlens)
+    long long kc0, kc1;   // packed key rows this chunk copies in (none an earlier chunk brought)
+};
+
+// Plan of the host-buffer pipeline.  Sequences are grouped whole until a
+// group holds about 1/kHostChunks of the query rows; a sequence longer than
+// that is cut into pieces of whole 256-row query blocks, each with the keys
+// its rows can see: the keys up to its last row's diagonal (causal, or a
+// window, which also bounds the keys from below, rounded down to a 128-key
+// tile) or all of the sequence's keys (neither).  The piece then computes
+// exactly what the whole sequence's launch computes for those rows: the same
+// query blocks, the same key tiles in the same order, the same masks (its
+// bottom-right diagonal offset is the sequence's, shifted by the keys left
+// out below), so the results are bit-identical.
+std::vector<HostChunk> plan_host_chunks(const int32_t* cu_q, const int32_t* cu_k, int batch, bool causal,
+                                        int window, size_t input_bytes) {
+    std::vector<HostChunk> out;
+    const long long T_q = cu_q[batch];
+    if (input_bytes < kHostChunkMinBytes || T_q == 0) {
+        out.push_back(HostChunk{false, 0, batch, 0, T_q, 0, 0, 0, cu_k[batch]});
+        return out;
+    }
+    const long long blk = va::kBlockQ;
+    const long long rows = std::max<long long>(kHostChunkMinRows,
+                                               (T_q + kHostChunks - 1) / kHostChunks + blk - 1) / blk * blk;
+    int g0 = 0;  // first sequence of the open group
+    auto close_group = [&](int b1) {
+        if (b1 > g0)
+            out.push_back(HostChunk{false, g0, b1, cu_q[g0], cu_q[b1], cu_k[g0], 0, cu_k[g0], cu_k[b1]});
+        g0 = b1;
+    };
+    for (int b = 0; b < batch; ++b) {
+        const long long L_q = cu_q[b + 1] - cu_q[b], L_k = cu_k[b + 1] - cu_k[b];
+        if (L_q <= rows) {
+            if (cu_q[b + 1] - cu_q[g0] >= rows) close_group(b + 1);
+            continue;
+        }
+        close_group(b);
+        const long long delta = L_k - L_q;
+        const bool banded = causal || window > 0;
+        long long copied = 0;  // keys of this sequence already copied in
+        for (long long r0 = 0; r0 < L_q; r0 += rows) {
+            const long long r1 = std::min(L_q, r0 + rows);
+            long long k_lo = 0, k_hi = L_k;
+            if (banded) {
+                k_hi = std::min(L_k, std::max(0ll, r1 + delta));
+                if (window > 0) k_lo = std::max(0ll, r0 + delta - window + 1) / va::kBlockN * va::kBlockN;
+                k_lo = std::min(k_lo, k_hi);
+            }
+            const long long c1 = std::max(copied, k_hi);
+            out.push_back(HostChunk{true, b, b + 1, cu_q[b] + r0, cu_q[b] + r1, cu_k[b] + k_lo, k_hi - k_lo,
+                                    cu_k[b] + copied, cu_k[b] + c1});
+            copied = c1;
+        }
+        g0 = b + 1;
+    }
+    close_group(batch);
+    return out;
+}
+
 }  // namespace
 
 extern "C" {
@@ -802,28 +871,28 @@ int varlen_attention_fwd_host(const void* q, const void* k, const void* v,
     const size_t qb = static_cast<size_t>(T_q) * q_row, kb = static_cast<size_t>(T_k) * k_row;
     const size_t ob = qb, lb = static_cast<size_t>(T_q) * l_row;
 
-    // Chunks of whole sequences, balanced by query tokens: chunk i's kernels
-    // run while chunk i + 1 is copied in and chunk i - 1 is copied out (the
-    // two directions on separate streams and copy engines).  Each sequence's
-    // result does not depend on which chunk or launch computes it.
-    std::vector<int> bounds{0};
-    const int n_want = (qb + 2 * kb >= kHostChunkMinBytes) ? std::min(kHostChunks, batch) : 1;
-    for (int c = 1; c < n_want; ++c) {
-        const long long target = T_q * c / n_want;
-        int b = bounds.back() + 1;
-        while (b < batch && cu_seqlens_q[b] < target) ++b;
-        if (b < batch) bounds.push_back(b);
-    }
-    bounds.push_back(batch);
-    const int n = static_cast<int>(bounds.size()) - 1;
-    // per chunk, cu_seqlens rebased to its first sequence (chunk c's arrays
-    // start at entry bounds[c] + c)
-    std::vector<int32_t> cu_h(2 * static_cast<size_t>(batch + n));
-    for (int c = 0; c < n; ++c)
-        for (int b = bounds[c]; b <= bounds[c + 1]; ++b) {
-            cu_h[b + c] = cu_seqlens_q[b] - cu_seqlens_q[bounds[c]];
-            cu_h[batch + n + b + c] = cu_seqlens_k[b] - cu_seqlens_k[bounds[c]];
+    // Chunks in packed query order: groups of whole sequences, and pieces of
+    // one long sequence (whole 256-row query blocks with the keys they can
+    // see).  Chunk i's kernels run while chunk i + 1 is copied in and chunk
+    // i - 1 is copied out (the two directions on separate streams and copy
+    // engines).
+    const std::vector<HostChunk> chunks =
+        plan_host_chunks(cu_seqlens_q, cu_seqlens_k, batch, causal != 0, window, qb + 2 * kb);
+    const int n = static_cast<int>(chunks.size());
+    // per chunk, cu_seqlens rebased to the chunk's first query row and first key
+    std::vector<int32_t> cu_h;
+    std::vector<size_t> cu_off(n);
+    for (int c = 0; c < n; ++c) {
+        const HostChunk& h = chunks[c];
+        cu_off[c] = cu_h.size();
+        if (h.piece) {
+            cu_h.insert(cu_h.end(), {0, static_cast<int32_t>(h.q1 - h.q0)});
+            cu_h.insert(cu_h.end(), {0, static_cast<int32_t>(h.k_len)});
+        } else {
+            for (int b = h.b0; b <= h.b1; ++b) cu_h.push_back(cu_seqlens_q[b] - cu_seqlens_q[h.b0]);
+            for (int b = h.b0; b <= h.b1; ++b) cu_h.push_back(cu_seqlens_k[b] - cu_seqlens_k[h.b0]);
         }
+    }
     const size_t cb = cu_h.size() * sizeof(int32_t);
 
     auto up256 = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
@@ -857,45 +926,45 @@ int varlen_attention_fwd_host(const void* q, const void* k, const void* v,
         if (e == cudaSuccess) e = cudaEventRecord(ev[0], stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev[0], 0);
     }
-    // every host-to-device copy, chunk after chunk, on the input stream
+    // every host-to-device copy, chunk after chunk, on the input stream: the
+    // chunk's query rows and the key rows it needs that no earlier chunk
+    // brought (a chunk's event so also covers every earlier copy)
     if (e == cudaSuccess && cb) e = cudaMemcpyAsync(dcu, cu_h.data(), cb, cudaMemcpyHostToDevice, s_in);
     for (int c = 0; c < n && e == cudaSuccess; ++c) {
-        const size_t r0 = cu_seqlens_q[bounds[c]], r1 = cu_seqlens_q[bounds[c + 1]];
-        const size_t k0 = cu_seqlens_k[bounds[c]], k1 = cu_seqlens_k[bounds[c + 1]];
-        if (r1 > r0)
-            e = cudaMemcpyAsync(dq + r0 * q_row, static_cast<const char*>(q) + r0 * q_row,
-                                (r1 - r0) * q_row, cudaMemcpyHostToDevice, s_in);
-        if (e == cudaSuccess && k1 > k0)
-            e = cudaMemcpyAsync(dk + k0 * k_row, static_cast<const char*>(k) + k0 * k_row,
-                                (k1 - k0) * k_row, cudaMemcpyHostToDevice, s_in);
-        if (e == cudaSuccess && k1 > k0)
-            e = cudaMemcpyAsync(dv + k0 * k_row, static_cast<const char*>(v) + k0 * k_row,
-                                (k1 - k0) * k_row, cudaMemcpyHostToDevice, s_in);
+        const HostChunk& h = chunks[c];
+        if (h.q1 > h.q0)
+            e = cudaMemcpyAsync(dq + h.q0 * q_row, static_cast<const char*>(q) + h.q0 * q_row,
+                                (h.q1 - h.q0) * q_row, cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess && h.kc1 > h.kc0)
+            e = cudaMemcpyAsync(dk + h.kc0 * k_row, static_cast<const char*>(k) + h.kc0 * k_row,
+                                (h.kc1 - h.kc0) * k_row, cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess && h.kc1 > h.kc0)
+            e = cudaMemcpyAsync(dv + h.kc0 * k_row, static_cast<const char*>(v) + h.kc0 * k_row,
+                                (h.kc1 - h.kc0) * k_row, cudaMemcpyHostToDevice, s_in);
         if (e == cudaSuccess && n > 1) e = cudaEventRecord(ev[1 + c], s_in);
     }
     // chunk by chunk: its kernels on the caller's stream, then its results
     // back on the output stream
     for (int c = 0; c < n && e == cudaSuccess && rc == VA_OK; ++c) {
-        const size_t r0 = cu_seqlens_q[bounds[c]], r1 = cu_seqlens_q[bounds[c + 1]];
-        const size_t k0 = cu_seqlens_k[bounds[c]];
+        const HostChunk& h = chunks[c];
         if (n > 1) e = cudaStreamWaitEvent(stream, ev[1 + c], 0);
         if (e != cudaSuccess) break;
-        Args d{dq + r0 * q_row, dk + k0 * k_row, dv + k0 * k_row, dcu + bounds[c] + c,
-               dcu + batch + n + bounds[c] + c, bounds[c + 1] - bounds[c], num_heads, num_kv_heads,
-               max_seqlen_q, max_seqlen_k, head_dim, causal ? 1 : 0, window, dout + r0 * q_row,
-               dlse + r0 * num_heads};
+        const int nb = h.piece ? 1 : h.b1 - h.b0;
+        Args d{dq + h.q0 * q_row, dk + h.k_base * k_row, dv + h.k_base * k_row, dcu + cu_off[c],
+               dcu + cu_off[c] + nb + 1, nb, num_heads, num_kv_heads, max_seqlen_q, max_seqlen_k,
+               head_dim, causal ? 1 : 0, window, dout + h.q0 * q_row, dlse + h.q0 * num_heads};
         rc = forward(d, VA_PATH_AUTO, 0, stream);
         if (rc != VA_OK) break;
         if (n > 1) {
             e = cudaEventRecord(ev[1 + n + c], stream);
             if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev[1 + n + c], 0);
         }
-        if (e == cudaSuccess && r1 > r0)
-            e = cudaMemcpyAsync(static_cast<char*>(out) + r0 * q_row, dout + r0 * q_row,
-                                (r1 - r0) * q_row, cudaMemcpyDeviceToHost, s_out);
-        if (e == cudaSuccess && r1 > r0)
-            e = cudaMemcpyAsync(reinterpret_cast<char*>(lse) + r0 * l_row,
-                                reinterpret_cast<char*>(dlse) + r0 * l_row, (r1 - r0) * l_row,
+        if (e == cudaSuccess && h.q1 > h.q0)
+            e = cudaMemcpyAsync(static_cast<char*>(out) + h.q0 * q_row, dout + h.q0 * q_row,
+                                (h.q1 - h.q0) * q_row, cudaMemcpyDeviceToHost, s_out);
+        if (e == cudaSuccess && h.q1 > h.q0)
+            e = cudaMemcpyAsync(reinterpret_cast<char*>(lse) + h.q0 * l_row,
+                                reinterpret_cast<char*>(dlse) + h.q0 * l_row, (h.q1 - h.q0) * l_row,
                                 cudaMemcpyDeviceToHost, s_out);
     }
     // the caller's stream waits for both copy streams (also after an error,
@@ -919,6 +988,31 @@ int varlen_attention_fwd_host(const void* q, const void* k, const void* v,
     if (rc != VA_OK) return rc;
     if (e != cudaSuccess) return cuda_fail(e, "host-buffer copies");
     if (se != cudaSuccess) return cuda_fail(se, "cudaStreamSynchronize");
+    return VA_OK;
+}
+
+int varlen_attention_host_chunks(const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int batch,
+                                 int causal, int window, long long input_bytes, long long* chunks,
+                                 int capacity, int* n_chunks) {
+    g_last_error[0] = 0;
+    if (!cu_seqlens_q || !cu_seqlens_k || !n_chunks)
+        return fail(VA_ERR_INVALID_ARG, "cu_seqlens_q, cu_seqlens_k and n_chunks must not be NULL");
+    if (batch < 0) return fail(VA_ERR_INVALID_ARG, "batch must be >= 0 (got %d)", batch);
+    if (window < 0) return fail(VA_ERR_INVALID_ARG, "window must be >= 0 (got %d)", window);
+    int rc;
+    if ((rc = check_cu_seqlens_host(cu_seqlens_q, batch, INT_MAX, -1, "cu_seqlens_q")) != VA_OK ||
+        (rc = check_cu_seqlens_host(cu_seqlens_k, batch, INT_MAX, -1, "cu_seqlens_k")) != VA_OK)
+        return rc;
+    const std::vector<HostChunk> plan = plan_host_chunks(
+        cu_seqlens_q, cu_seqlens_k, batch, causal != 0, window, static_cast<size_t>(std::max(0ll, input_bytes)));
+    *n_chunks = static_cast<int>(plan.size());
+    if (static_cast<int>(plan.size()) > capacity || (!chunks && !plan.empty()))
+        return fail(VA_ERR_INVALID_ARG, "capacity %d below the %zu chunks of the plan", capacity, plan.size());
+    for (size_t c = 0; c < plan.size(); ++c) {
+        const HostChunk& h = plan[c];
+        const long long f[9] = {h.piece ? 1 : 0, h.b0, h.b1, h.q0, h.q1, h.k_base, h.k_len, h.kc0, h.kc1};
+        std::copy(f, f + 9, chunks + 9 * c);
+    }
     return VA_OK;
 }
 
