@@ -25,8 +25,9 @@
 //                      dV += P^T dout runs, then dK += dS^T Q (TS form), the
 //                      two accumulators in tensor memory over the whole loop
 // An item's resident tiles are reloaded once its last products that read them
-// are done, its accumulators read out by the element-wise warps before the
-// next item's first product overwrites them; the products of one item's steps
+// (its last S and dP, issued first in its last step) are done, its
+// accumulators read out by the element-wise warps before the next item's
+// first product overwrites them; the products of one item's steps
 // and the barrier phases run on across items.
 // Warp roles (320 threads): warps 0-7 the element-wise work and the epilogue
 // (one key row, or one query row, per thread; warps w and w + 4 share a
@@ -312,19 +313,20 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
             for (int n = 0; n < n_steps; ++n, ++ring_n) {
                 const int st = ring_n & 1;
                 const int h = hk * G + n / n_qt, qt = qt0 + n % n_qt;
+                // the tile's 128 rows of {lse * log2(e), Delta} (written by the dQ
+                // kernel), four loads per lane in flight while the stage drains
+                // (rows past the sequence are masked: any finite value)
+                const float2* src = p.rowinfo + h * p.rows_cap + cq + qt * kBlockM;
+                float2 ri[kBlockM / 32];
+#pragma unroll
+                for (int u = 0; u < kBlockM / 32; ++u) {
+                    const int r = lane + 32 * u;
+                    ri[u] = qt * kBlockM + r < L_q ? src[r] : make_float2(0.f, 0.f);
+                }
                 if (!(ok = mbar_wait_warp(&bar.ring_empty[st], ((ring_n >> 1) & 1) ^ 1, bar.abort_flag, status)))
                     break;
                 {
-                    // the tile's 128 rows of {lse * log2(e), Delta}, staged negated (the
-                    // element-wise warps add them): four loads per lane in flight at once
-                    // (rows past the sequence are masked: any finite value)
-                    const float2* src = p.rowinfo + h * p.rows_cap + cq + qt * kBlockM;
-                    float2 ri[kBlockM / 32];
-#pragma unroll
-                    for (int u = 0; u < kBlockM / 32; ++u) {
-                        const int r = lane + 32 * u;
-                        ri[u] = qt * kBlockM + r < L_q ? src[r] : make_float2(0.f, 0.f);
-                    }
+                    // staged negated (the element-wise warps add them)
 #pragma unroll
                     for (int u = 0; u < kBlockM / 32; ++u) {
                         lse_s[st * kBlockM + lane + 32 * u] = -ri[u].x;
@@ -402,6 +404,10 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                                             static_cast<uint32_t>(dd_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(bar.dp_full);
+                    // the item's last products that read K and V (its last S^T and dP^T)
+                    // are issued: the next item's K and V may load while this step's
+                    // dV and dK run
+                    if (n + 1 == n_steps) mma_commit(bar.fixed_empty);
                     if (!(ok = mbar_wait(bar.p_ready, m & 1, bar.abort_flag, status))) break;
                     // the first dV of an item overwrites the accumulators: the previous
                     // item's must have been read out
@@ -434,7 +440,6 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                     mma_commit(&bar.ring_empty[st]);
                 }
                 if (!ok) break;
-                mma_commit(bar.fixed_empty);  // K and V may be reloaded
                 mma_commit(bar.acc_done);
                 g += n_steps;
                 ++acc_n;
@@ -751,6 +756,9 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                                             static_cast<uint32_t>(dv_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(bar.dp_full);
+                    // the item's last products that read Q and dout (its last S and dP)
+                    // are issued: the next item's Q and dout may load while dQ runs
+                    if (n + 1 == n_steps) mma_commit(bar.fixed_empty);
                     if (n + 1 < n_steps) {
                         if (!(ok = mbar_wait(&bar.ring_full[(m + 1) & 1], ((m + 1) >> 1) & 1, bar.abort_flag,
                                              status)))
@@ -776,7 +784,6 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                     mma_commit(&bar.ring_empty[st]);
                 }
                 if (!ok) break;
-                mma_commit(bar.fixed_empty);  // Q and dout may be reloaded
                 mma_commit(bar.acc_done);
                 g += n_steps;
                 ++acc_n;
