@@ -97,21 +97,26 @@ struct BwdMaps {
     CUtensorMap q8, dout8, k8, v8;
 };
 
-template <int D>
+template <int D, bool kDq>
 struct BwdSmem {
     using T = PrefillSmem<D, ElemBf16>;
     static constexpr int kTile = T::kTileBytes;  // 128 rows x D bf16, 128-byte swizzle
-    // dK/dV kernel: K, V once; Q, dout, base-2 lse and Delta double-buffered
-    // dQ kernel:   Q, dout once; K, V double-buffered
+    // dK/dV kernel: K, V once; Q (ring 0) and dout (ring 1) double-buffered, with
+    //               the base-2 lse and Delta of each Q stage
+    // dQ kernel:   Q, dout once; K in a three-stage ring (ring 0: its last reader,
+    //               dQ, ends the step, and the next-but-one step's S starts the
+    //               next), V double-buffered (ring 1: read by dP only, early)
+    static constexpr int kStages0 = kDq ? 3 : 2;
     static constexpr int kFixed0 = 0;
     static constexpr int kFixed1 = kTile;
-    static constexpr int kRing0 = 2 * kTile;      // [2]
-    static constexpr int kRing1 = 4 * kTile;      // [2]
-    static constexpr int kRows = 6 * kTile;       // [2][128] f32 lse * log2(e), [2][128] f32 Delta
-    static constexpr int kBar = kRows + 4 * 128 * 4;
-    // fixed_full, ring_full[2], ring_empty[2], s_full, p_ready, acc_done, dp_full, ds_ready,
-    // p_read, fixed_empty, acc_free, item_full[2], item_empty[2]
-    static constexpr int kNumBars = 17;
+    static constexpr int kRing0 = 2 * kTile;                  // [kStages0]
+    static constexpr int kRing1 = kRing0 + kStages0 * kTile;  // [2]
+    static constexpr int kRows = kRing1 + 2 * kTile;          // dK/dV: [2][128] f32 lse * log2(e), [2][128] f32 Delta
+    static constexpr int kBar = kRows + (kDq ? 0 : 4 * 128 * 4);
+    // fixed_full, ring_full[3], ring_empty[3], s_full, p_ready, acc_done, dp_full, ds_ready,
+    // p_read, fixed_empty, acc_free, item_full[2], item_empty[2], ring1_full[2], ring1_empty[2]
+    // (the dK/dV kernel's rings share ring_full / ring_empty, two stages)
+    static constexpr int kNumBars = 23;
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag
     static constexpr int kItems = kMisc + 16;          // BwdItem [2]
     static constexpr int kBytes = kItems + 2 * 32;
@@ -122,8 +127,10 @@ struct BwdSmem {
 // Per-role state shared by the two tile kernels.
 struct BwdBars {
     uint64_t* fixed_full;
-    uint64_t* ring_full;   // [2]
-    uint64_t* ring_empty;  // [2]
+    uint64_t* ring_full;   // [kStages0]: ring 0 (and ring 1 in the dK/dV kernel) loaded
+    uint64_t* ring_empty;  // [kStages0]
+    uint64_t* ring1_full;   // [2]: dQ kernel, V loaded
+    uint64_t* ring1_empty;  // [2]
     uint64_t* s_full;
     uint64_t* p_ready;
     uint64_t* acc_done;
@@ -139,32 +146,38 @@ struct BwdBars {
     BwdItem* items;         // [2]
 };
 
-template <int D>
+template <int D, bool kDq>
 __device__ __forceinline__ BwdBars bwd_setup(uint8_t* smem, int warp) {
-    using L = BwdSmem<D>;
+    using L = BwdSmem<D, kDq>;
     BwdBars r;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
     r.fixed_full = bars;
     r.ring_full = bars + 1;
-    r.ring_empty = bars + 3;
-    r.s_full = bars + 5;
-    r.p_ready = bars + 6;
-    r.acc_done = bars + 7;
-    r.dp_full = bars + 8;
-    r.ds_ready = bars + 9;
-    r.p_read = bars + 10;
-    r.fixed_empty = bars + 11;
-    r.acc_free = bars + 12;
-    r.item_full = bars + 13;
-    r.item_empty = bars + 15;
+    r.ring_empty = bars + 4;
+    r.s_full = bars + 7;
+    r.p_ready = bars + 8;
+    r.acc_done = bars + 9;
+    r.dp_full = bars + 10;
+    r.ds_ready = bars + 11;
+    r.p_read = bars + 12;
+    r.fixed_empty = bars + 13;
+    r.acc_free = bars + 14;
+    r.item_full = bars + 15;
+    r.item_empty = bars + 17;
+    r.ring1_full = bars + 19;
+    r.ring1_empty = bars + 21;
     r.tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     r.abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     r.items = reinterpret_cast<BwdItem*>(smem + L::kItems);
     if (threadIdx.x == 0) {
         mbar_init(r.fixed_full, 2);  // two tile loads
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&r.ring_full[s], 2);
+        for (int s = 0; s < L::kStages0; ++s) {
+            mbar_init(&r.ring_full[s], kDq ? 1 : 2);  // K alone, or Q and dout
             mbar_init(&r.ring_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&r.ring1_full[s], 1);
+            mbar_init(&r.ring1_empty[s], 1);
         }
         mbar_init(r.s_full, 1);
         mbar_init(r.p_ready, kBwdEwWarps);
@@ -242,7 +255,7 @@ __device__ __forceinline__ void bwd_store_rows(uint32_t taddr, float mul, uint8_
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
-    using L = BwdSmem<D>;
+    using L = BwdSmem<D, false>;
     using T = PrefillSmem<D, ElemBf16>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -250,7 +263,7 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.H / p.H_kv;
     const long long kv_pitch = static_cast<long long>(p.H_kv) * D * 2;
-    const BwdBars bar = bwd_setup<D>(smem, warp);
+    const BwdBars bar = bwd_setup<D, false>(smem, warp);
     const uint32_t tmem = *bar.tmem_slot;
     unsigned* status = &g_va_status;
     float* lse_s = reinterpret_cast<float*>(smem + L::kRows);            // [2][128]
@@ -631,13 +644,13 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
-    using L = BwdSmem<D>;
+    using L = BwdSmem<D, true>;
     using T = PrefillSmem<D, ElemBf16>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const BwdBars bar = bwd_setup<D>(smem, warp);
+    const BwdBars bar = bwd_setup<D, true>(smem, warp);
     const uint32_t tmem = *bar.tmem_slot;
     unsigned* status = &g_va_status;
     constexpr uint32_t kS = 0, kDP = 128, kDQ = 256;  // tensor-memory columns
@@ -649,7 +662,7 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
         // ------------------------------------------------------------ producer
         const int T_q = p.cu_q[p.batch], T_k = p.cu_k[p.batch];
         const int q_stride = p.H * D * 2, kv_stride = p.H_kv * D * 2;
-        uint32_t ring_n = 0, fixed_n = 0, item_n = 0, issued[2] = {0, 0};
+        uint32_t ring_n = 0, fixed_n = 0, item_n = 0, issued_k[3] = {0, 0, 0}, issued_v[2] = {0, 0};
         bool ok = true;
         for (;;) {
             // claim the next item (longest first across the grid) and publish it
@@ -686,22 +699,28 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                                    h * D, bar.fixed_full, lane);
             ++fixed_n;
             for (int n = 0; n < n_steps; ++n, ++ring_n) {
-                const int st = ring_n & 1, kt = it.a0 + n;
-                if (!(ok = mbar_wait_warp(&bar.ring_empty[st], ((ring_n >> 1) & 1) ^ 1, bar.abort_flag, status)))
+                // K into stage ring_n % 3 of ring 0, V into stage ring_n % 2 of ring 1
+                const int sk = static_cast<int>(ring_n % L::kStages0), sv = ring_n & 1, kt = it.a0 + n;
+                if (!(ok = mbar_wait_warp(&bar.ring_empty[sk], ((ring_n / L::kStages0) & 1) ^ 1, bar.abort_flag,
+                                          status)))
                     break;
-                load_tile<D, ElemBf16>(smem + L::kRing0 + st * L::kTile, &maps.k, &maps.k8, p.k,
-                                       ck + kt * kBlockN, T_k, kv_stride, hk * D, &bar.ring_full[st], lane);
-                load_tile<D, ElemBf16>(smem + L::kRing1 + st * L::kTile, &maps.v, &maps.v8, p.v,
-                                       ck + kt * kBlockN, T_k, kv_stride, hk * D, &bar.ring_full[st], lane);
-                ++issued[st];
+                load_tile<D, ElemBf16>(smem + L::kRing0 + sk * L::kTile, &maps.k, &maps.k8, p.k,
+                                       ck + kt * kBlockN, T_k, kv_stride, hk * D, &bar.ring_full[sk], lane);
+                ++issued_k[sk];
+                if (!(ok = mbar_wait_warp(&bar.ring1_empty[sv], ((ring_n >> 1) & 1) ^ 1, bar.abort_flag, status)))
+                    break;
+                load_tile<D, ElemBf16>(smem + L::kRing1 + sv * L::kTile, &maps.v, &maps.v8, p.v,
+                                       ck + kt * kBlockN, T_k, kv_stride, hk * D, &bar.ring1_full[sv], lane);
+                ++issued_v[sv];
             }
             if (!ok) break;
         }
         if (!ok && lane == 0) {
             const unsigned long long t0 = global_timer_ns();
             bwd_drain(bar.fixed_full, fixed_n, t0);
-            bwd_drain(&bar.ring_full[0], issued[0], t0);
-            bwd_drain(&bar.ring_full[1], issued[1], t0);
+            for (int sk = 0; sk < L::kStages0; ++sk) bwd_drain(&bar.ring_full[sk], issued_k[sk], t0);
+            bwd_drain(&bar.ring1_full[0], issued_v[0], t0);
+            bwd_drain(&bar.ring1_full[1], issued_v[1], t0);
         }
     } else if (warp == kBwdMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -714,9 +733,9 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
             const uint64_t dv_k = smem_desc_sw128(smem_u32(smem + L::kRing1), 16, 1024);
             const uint64_t dk_mn = smem_desc_sw128(smem_u32(smem + L::kRing0), T::kChunkBytes, 1024);
             const uint32_t hi_k = static_cast<uint32_t>(dq_ >> 32), hi_mn = static_cast<uint32_t>(dk_mn >> 32);
-            // S = Q K^T for step m (K of ring stage m & 1, K-major operands, K = D)
+            // S = Q K^T for step m (K of ring-0 stage m % 3, K-major operands, K = D)
             auto issue_s = [&](uint32_t m) {
-                const uint32_t ring = ((m & 1) * L::kTile) >> 4;
+                const uint32_t ring = ((m % L::kStages0) * L::kTile) >> 4;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * T::kChunkBytes + (kk & 3) * 32) >> 4;
@@ -738,30 +757,36 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                 if (n_steps <= 0) continue;
                 if (!(ok = mbar_wait(bar.fixed_full, fixed_n & 1, bar.abort_flag, status))) break;
                 ++fixed_n;
-                if (!(ok = mbar_wait(&bar.ring_full[g & 1], (g >> 1) & 1, bar.abort_flag, status))) break;
+                if (!(ok = mbar_wait(&bar.ring_full[g % L::kStages0], (g / L::kStages0) & 1, bar.abort_flag,
+                                     status)))
+                    break;
                 tc_fence_after();
                 issue_s(g);
                 // Order per step m: dP(m), S(m+1) once the element-wise warps have read
                 // S(m), dQ(m) once dS(m) is stored.  The next S so runs while dS is
-                // formed; dP(m+1) overwrites dS(m) and follows dQ(m).
+                // formed; dP(m+1) overwrites dS(m) and follows dQ(m).  V(m) is
+                // released as soon as dP(m) completes, K(m) once dQ(m) does.
                 for (int n = 0; n < n_steps && ok; ++n) {
                     const uint32_t m = g + n;
-                    const int st = m & 1;
-                    const uint32_t ring = (st * L::kTile) >> 4;
+                    const int sk = static_cast<int>(m % L::kStages0), sv = m & 1;
+                    const uint32_t ring_k = (sk * L::kTile) >> 4, ring_v = (sv * L::kTile) >> 4;
+                    if (!(ok = mbar_wait(&bar.ring1_full[sv], (m >> 1) & 1, bar.abort_flag, status))) break;
+                    tc_fence_after();
                     // dP = dout V^T (K-major operands, K = D)
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t off = ((kk >> 2) * T::kChunkBytes + (kk & 3) * 32) >> 4;
                         mma_ss_lh<idesc_ss>(tmem + kDP, static_cast<uint32_t>(dd_) + off, hi_k,
-                                            static_cast<uint32_t>(dv_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
+                                            static_cast<uint32_t>(dv_k) + ring_v + off, hi_k, kk > 0 ? 1u : 0u);
                     }
                     mma_commit(bar.dp_full);
+                    mma_commit(&bar.ring1_empty[sv]);
                     // the item's last products that read Q and dout (its last S and dP)
                     // are issued: the next item's Q and dout may load while dQ runs
                     if (n + 1 == n_steps) mma_commit(bar.fixed_empty);
                     if (n + 1 < n_steps) {
-                        if (!(ok = mbar_wait(&bar.ring_full[(m + 1) & 1], ((m + 1) >> 1) & 1, bar.abort_flag,
-                                             status)))
+                        if (!(ok = mbar_wait(&bar.ring_full[(m + 1) % L::kStages0], ((m + 1) / L::kStages0) & 1,
+                                             bar.abort_flag, status)))
                             break;
                         if (!(ok = mbar_wait(bar.p_read, m & 1, bar.abort_flag, status))) break;
                         tc_fence_after();
@@ -778,10 +803,10 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
 #pragma unroll
                     for (int kk = 0; kk < kBlockN / 16; ++kk) {
                         mma_ts_lh<idesc_ts>(tmem + kDQ, tmem + kDP + bwd_kcol(kk),
-                                            static_cast<uint32_t>(dk_mn) + ring + ((kk * 16 * 128) >> 4), hi_mn,
+                                            static_cast<uint32_t>(dk_mn) + ring_k + ((kk * 16 * 128) >> 4), hi_mn,
                                             (n > 0 || kk > 0) ? 1u : 0u);
                     }
-                    mma_commit(&bar.ring_empty[st]);
+                    mma_commit(&bar.ring_empty[sk]);
                 }
                 if (!ok) break;
                 mma_commit(bar.acc_done);

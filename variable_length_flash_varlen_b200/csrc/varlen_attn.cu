@@ -130,13 +130,13 @@ int device_setup(int& dev, DeviceInfo*& info) {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  va::kSortCapacity * 8));
     VA_CUDA(cudaFuncSetAttribute(va::bwd_dkdv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::BwdSmem<64>::kAlloc));
+                                 va::BwdSmem<64, false>::kAlloc));
     VA_CUDA(cudaFuncSetAttribute(va::bwd_dkdv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::BwdSmem<128>::kAlloc));
+                                 va::BwdSmem<128, false>::kAlloc));
     VA_CUDA(cudaFuncSetAttribute(va::bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::BwdSmem<64>::kAlloc));
+                                 va::BwdSmem<64, true>::kAlloc));
     VA_CUDA(cudaFuncSetAttribute(va::bwd_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 va::BwdSmem<128>::kAlloc));
+                                 va::BwdSmem<128, true>::kAlloc));
     VA_CUDA(cudaFuncSetAttribute(va::decode_stream_kernel<64>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  va::DecodeSmem<64>::kAlloc));
@@ -590,14 +590,14 @@ int run_backward(const BwdArgs& g, cudaStream_t stream) {
     const int grid_q = static_cast<int>(std::min<long long>(info->num_sms, cap_q_ll * a.H));
     const int grid_kv = static_cast<int>(std::min<long long>(info->num_sms, cap_k_ll * a.H_kv));
     if (a.D == 64) {
-        if (grid_q > 0) va::bwd_dq_kernel<64><<<grid_q, va::kBwdThreads, va::BwdSmem<64>::kAlloc, stream>>>(maps, p);
+        if (grid_q > 0) va::bwd_dq_kernel<64><<<grid_q, va::kBwdThreads, va::BwdSmem<64, true>::kAlloc, stream>>>(maps, p);
         if (grid_kv > 0)
-            va::bwd_dkdv_kernel<64><<<grid_kv, va::kBwdThreads, va::BwdSmem<64>::kAlloc, stream>>>(maps, p);
+            va::bwd_dkdv_kernel<64><<<grid_kv, va::kBwdThreads, va::BwdSmem<64, false>::kAlloc, stream>>>(maps, p);
     } else {
         if (grid_q > 0)
-            va::bwd_dq_kernel<128><<<grid_q, va::kBwdThreads, va::BwdSmem<128>::kAlloc, stream>>>(maps, p);
+            va::bwd_dq_kernel<128><<<grid_q, va::kBwdThreads, va::BwdSmem<128, true>::kAlloc, stream>>>(maps, p);
         if (grid_kv > 0)
-            va::bwd_dkdv_kernel<128><<<grid_kv, va::kBwdThreads, va::BwdSmem<128>::kAlloc, stream>>>(maps, p);
+            va::bwd_dkdv_kernel<128><<<grid_kv, va::kBwdThreads, va::BwdSmem<128, false>::kAlloc, stream>>>(maps, p);
     }
     cudaError_t le = cudaGetLastError();
     cudaFreeAsync(ws, stream);
