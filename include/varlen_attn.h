@@ -63,6 +63,7 @@ extern "C" {
 /* Device status bits (varlen_attention_device_status). */
 #define VA_STATUS_WAIT_TIMEOUT 1u       /* a bounded wait inside a kernel gave up */
 #define VA_STATUS_SCHEDULE_OVERFLOW 2u  /* more query tiles than max_seqlen_q allows for */
+#define VA_STATUS_SMEM_ALIGN 4u         /* a backward kernel found its shared memory misaligned and did nothing */
 
 /* Path selection for varlen_attention_fwd_ex. */
 #define VA_PATH_AUTO 0    /* decode when max_seqlen_q == 1, else prefill */
@@ -275,7 +276,9 @@ int varlen_attention_device_status(unsigned* status, int clear);
  * here too once that work has finished.
  * Returns VA_ERR_DEVICE_TIMEOUT when VA_STATUS_WAIT_TIMEOUT is set (a
  * kernel's bounded wait gave up: its results are incomplete),
- * VA_ERR_INVALID_ARG when only VA_STATUS_SCHEDULE_OVERFLOW is set (a query
+ * VA_ERR_CUDA when VA_STATUS_SMEM_ALIGN is set (a kernel that fills nearly all
+ * of a CTA's shared memory found its base not 1024-byte aligned and wrote
+ * nothing), VA_ERR_INVALID_ARG when only VA_STATUS_SCHEDULE_OVERFLOW is set (a query
  * length exceeded max_seqlen_q), VA_OK when the word is 0; VA_ERR_CUDA if a
  * copy or the synchronisation fails, VA_ERR_INVALID_ARG for a NULL status.
  * It blocks the calling host thread until `stream` drains, so it must not be

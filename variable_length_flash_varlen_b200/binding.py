@@ -21,6 +21,7 @@ VA_ERR_INVALID_ARG, VA_ERR_UNSUPPORTED, VA_ERR_CUDA, VA_ERR_DEVICE_TIMEOUT = -1,
 VA_PATH_AUTO, VA_PATH_PREFILL, VA_PATH_DECODE = 0, 1, 2
 VA_STATUS_WAIT_TIMEOUT = 1
 VA_STATUS_SCHEDULE_OVERFLOW = 2
+VA_STATUS_SMEM_ALIGN = 4
 
 # every symbol the header declares, with its ctypes signature
 _P, _I = ctypes.c_void_p, ctypes.c_int

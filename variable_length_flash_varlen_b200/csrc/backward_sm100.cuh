@@ -20,10 +20,11 @@
 //   bwd_dkdv_kernel    item = (key tile of 128 keys, KV head, sequence):
 //                      K and V stay in shared memory; for every query head of
 //                      the group and every 128-row query tile that sees the key
-//                      tile: S^T = K Q^T, then P^T (bf16) into tensor memory
-//                      while dP^T = V dout^T runs, then dS^T (bf16) while
-//                      dV += P^T dout runs, then dK += dS^T Q (TS form), the
-//                      two accumulators in tensor memory over the whole loop
+//                      tile: S^T = K Q^T, P^T (bf16, in registers) while dP^T =
+//                      V dout^T runs, then dS^T, both stored (bf16) over the dP^T
+//                      columns, then dV += P^T dout and dK += dS^T Q (TS form),
+//                      the two accumulators in tensor memory over the whole
+//                      loop; the next S^T runs as soon as S^T has been read
 // An item's resident tiles are reloaded once its last products that read them
 // (its last S and dP, issued first in its last step) are done, its
 // accumulators read out by the element-wise warps before the next item's
@@ -101,12 +102,13 @@ template <int D, bool kDq>
 struct BwdSmem {
     using T = PrefillSmem<D, ElemBf16>;
     static constexpr int kTile = T::kTileBytes;  // 128 rows x D bf16, 128-byte swizzle
-    // dK/dV kernel: K, V once; Q (ring 0) and dout (ring 1) double-buffered, with
-    //               the base-2 lse and Delta of each Q stage
-    // dQ kernel:   Q, dout once; K in a three-stage ring (ring 0: its last reader,
-    //               dQ, ends the step, and the next-but-one step's S starts the
-    //               next), V double-buffered (ring 1: read by dP only, early)
-    static constexpr int kStages0 = kDq ? 3 : 2;
+    // Ring 0 has three stages: its tile's last reader (dQ, or dK) ends a step
+    // while the next-but-one step's first product (S, or S^T) starts the next.
+    // dK/dV kernel: K, V once; Q in ring 0; dout in ring 1 (two stages) with
+    //               the base-2 lse and Delta of its step
+    // dQ kernel:   Q, dout once; K in ring 0; V in ring 1 (two stages: read by
+    //               dP only, early in a step)
+    static constexpr int kStages0 = 3;
     static constexpr int kFixed0 = 0;
     static constexpr int kFixed1 = kTile;
     static constexpr int kRing0 = 2 * kTile;                  // [kStages0]
@@ -115,21 +117,26 @@ struct BwdSmem {
     static constexpr int kBar = kRows + (kDq ? 0 : 4 * 128 * 4);
     // fixed_full, ring_full[3], ring_empty[3], s_full, p_ready, acc_done, dp_full, ds_ready,
     // p_read, fixed_empty, acc_free, item_full[2], item_empty[2], ring1_full[2], ring1_empty[2]
-    // (the dK/dV kernel's rings share ring_full / ring_empty, two stages)
     static constexpr int kNumBars = 23;
     static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag
     static constexpr int kItems = kMisc + 16;          // BwdItem [2]
     static constexpr int kBytes = kItems + 2 * 32;
-    static constexpr int kAlloc = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
+    // 1 KB of slack aligns the layout to 1024 bytes inside any base; a layout
+    // too large for the slack relies on the base itself being aligned (the
+    // kernel checks, and on a misaligned base raises kStatusSmemAlign and
+    // returns before any access)
+    static constexpr bool kNeedsAlignedBase = kBytes + 1024 > 232448;
+    static constexpr int kAlloc =
+        kNeedsAlignedBase ? kBytes : ((kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024);
     static_assert(kAlloc <= 232448, "beyond the 227 KB of shared memory a CTA may use");
 };
 
 // Per-role state shared by the two tile kernels.
 struct BwdBars {
     uint64_t* fixed_full;
-    uint64_t* ring_full;   // [kStages0]: ring 0 (and ring 1 in the dK/dV kernel) loaded
-    uint64_t* ring_empty;  // [kStages0]
-    uint64_t* ring1_full;   // [2]: dQ kernel, V loaded
+    uint64_t* ring_full;    // [kStages0]: ring 0 (K or Q) loaded
+    uint64_t* ring_empty;   // [kStages0]
+    uint64_t* ring1_full;   // [2]: ring 1 (V, or dout and its step's lse / Delta) loaded
     uint64_t* ring1_empty;  // [2]
     uint64_t* s_full;
     uint64_t* p_ready;
@@ -172,7 +179,7 @@ __device__ __forceinline__ BwdBars bwd_setup(uint8_t* smem, int warp) {
     if (threadIdx.x == 0) {
         mbar_init(r.fixed_full, 2);  // two tile loads
         for (int s = 0; s < L::kStages0; ++s) {
-            mbar_init(&r.ring_full[s], kDq ? 1 : 2);  // K alone, or Q and dout
+            mbar_init(&r.ring_full[s], 1);  // one tile: K (dQ) or Q (dK/dV)
             mbar_init(&r.ring_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -260,6 +267,12 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
+    if constexpr (L::kNeedsAlignedBase) {
+        if (smem != smem_raw) {  // uniform across the CTA: every thread leaves here
+            if (threadIdx.x == 0) atomicOr(&g_va_status, kStatusSmemAlign);
+            return;
+        }
+    }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.H / p.H_kv;
     const long long kv_pitch = static_cast<long long>(p.H_kv) * D * 2;
@@ -285,7 +298,7 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
         // ------------------------------------------------------------ producer
         const int T_q = p.cu_q[p.batch], T_k = p.cu_k[p.batch];
         const int q_stride = p.H * D * 2, kv_stride = p.H_kv * D * 2;
-        uint32_t ring_n = 0, fixed_n = 0, item_n = 0, issued[2] = {0, 0};
+        uint32_t ring_n = 0, fixed_n = 0, item_n = 0, issued_q[3] = {0, 0, 0}, issued_d[2] = {0, 0};
         bool ok = true;
         for (;;) {
             int idx = -1;
@@ -324,10 +337,12 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                                    hk * D, bar.fixed_full, lane);
             ++fixed_n;
             for (int n = 0; n < n_steps; ++n, ++ring_n) {
-                const int st = ring_n & 1;
+                // Q into stage ring_n % 3 of ring 0; dout and the step's lse / Delta
+                // rows into stage ring_n % 2 of ring 1
+                const int sq = static_cast<int>(ring_n % L::kStages0), sd = ring_n & 1;
                 const int h = hk * G + n / n_qt, qt = qt0 + n % n_qt;
                 // the tile's 128 rows of {lse * log2(e), Delta} (written by the dQ
-                // kernel), four loads per lane in flight while the stage drains
+                // kernel), four loads per lane in flight while the stages drain
                 // (rows past the sequence are masked: any finite value)
                 const float2* src = p.rowinfo + h * p.rows_cap + cq + qt * kBlockM;
                 float2 ri[kBlockM / 32];
@@ -336,30 +351,34 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                     const int r = lane + 32 * u;
                     ri[u] = qt * kBlockM + r < L_q ? src[r] : make_float2(0.f, 0.f);
                 }
-                if (!(ok = mbar_wait_warp(&bar.ring_empty[st], ((ring_n >> 1) & 1) ^ 1, bar.abort_flag, status)))
+                if (!(ok = mbar_wait_warp(&bar.ring_empty[sq], ((ring_n / L::kStages0) & 1) ^ 1, bar.abort_flag,
+                                          status)))
                     break;
-                {
-                    // staged negated (the element-wise warps add them)
+                load_tile<D, ElemBf16>(smem + L::kRing0 + sq * L::kTile, &maps.q, &maps.q8, p.q,
+                                       cq + qt * kBlockM, T_q, q_stride, h * D, &bar.ring_full[sq], lane);
+                ++issued_q[sq];
+                if (!(ok = mbar_wait_warp(&bar.ring1_empty[sd], ((ring_n >> 1) & 1) ^ 1, bar.abort_flag, status)))
+                    break;
+                // staged negated (the element-wise warps add them); released with
+                // the dout tile's arrival on ring1_full
 #pragma unroll
-                    for (int u = 0; u < kBlockM / 32; ++u) {
-                        lse_s[st * kBlockM + lane + 32 * u] = -ri[u].x;
-                        dlt_s[st * kBlockM + lane + 32 * u] = -ri[u].y;
-                    }
+                for (int u = 0; u < kBlockM / 32; ++u) {
+                    lse_s[sd * kBlockM + lane + 32 * u] = -ri[u].x;
+                    dlt_s[sd * kBlockM + lane + 32 * u] = -ri[u].y;
                 }
                 __syncwarp();
-                load_tile<D, ElemBf16>(smem + L::kRing0 + st * L::kTile, &maps.q, &maps.q8, p.q,
-                                       cq + qt * kBlockM, T_q, q_stride, h * D, &bar.ring_full[st], lane);
-                load_tile<D, ElemBf16>(smem + L::kRing1 + st * L::kTile, &maps.dout, &maps.dout8, p.dout,
-                                       cq + qt * kBlockM, T_q, q_stride, h * D, &bar.ring_full[st], lane);
-                ++issued[st];
+                load_tile<D, ElemBf16>(smem + L::kRing1 + sd * L::kTile, &maps.dout, &maps.dout8, p.dout,
+                                       cq + qt * kBlockM, T_q, q_stride, h * D, &bar.ring1_full[sd], lane);
+                ++issued_d[sd];
             }
             if (!ok) break;
         }
         if (!ok && lane == 0) {
             const unsigned long long t0 = global_timer_ns();
             bwd_drain(bar.fixed_full, fixed_n, t0);
-            bwd_drain(&bar.ring_full[0], issued[0], t0);
-            bwd_drain(&bar.ring_full[1], issued[1], t0);
+            for (int sq = 0; sq < L::kStages0; ++sq) bwd_drain(&bar.ring_full[sq], issued_q[sq], t0);
+            bwd_drain(&bar.ring1_full[0], issued_d[0], t0);
+            bwd_drain(&bar.ring1_full[1], issued_d[1], t0);
         }
     } else if (warp == kBwdMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -373,9 +392,9 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
             const uint64_t dq_mn = smem_desc_sw128(smem_u32(smem + L::kRing0), T::kChunkBytes, 1024);
             const uint64_t dd_mn = smem_desc_sw128(smem_u32(smem + L::kRing1), T::kChunkBytes, 1024);
             const uint32_t hi_k = static_cast<uint32_t>(dk_ >> 32), hi_mn = static_cast<uint32_t>(dq_mn >> 32);
-            // S^T = K Q^T for step m (Q of ring stage m & 1, K-major operands, K = D)
+            // S^T = K Q^T for step m (Q of ring-0 stage m % 3, K-major operands, K = D)
             auto issue_s = [&](uint32_t m) {
-                const uint32_t ring = ((m & 1) * L::kTile) >> 4;
+                const uint32_t ring = ((m % L::kStages0) * L::kTile) >> 4;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * T::kChunkBytes + (kk & 3) * 32) >> 4;
@@ -383,6 +402,17 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                                         static_cast<uint32_t>(dq_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar.s_full);
+            };
+            // dP^T = V dout^T for step m (dout of ring-1 stage m & 1, K-major operands, K = D)
+            auto issue_dp = [&](uint32_t m) {
+                const uint32_t ring = ((m & 1) * L::kTile) >> 4;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * T::kChunkBytes + (kk & 3) * 32) >> 4;
+                    mma_ss_lh<idesc_ss>(tmem + kDP, static_cast<uint32_t>(dv_) + off, hi_k,
+                                        static_cast<uint32_t>(dd_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar.dp_full);
             };
             uint32_t g = 0, fixed_n = 0, acc_n = 0, item_n = 0;
             bool ok = true;
@@ -397,60 +427,63 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                 if (n_steps == 0) continue;
                 if (!(ok = mbar_wait(bar.fixed_full, fixed_n & 1, bar.abort_flag, status))) break;
                 ++fixed_n;
-                if (!(ok = mbar_wait(&bar.ring_full[g & 1], (g >> 1) & 1, bar.abort_flag, status))) break;
+                if (!(ok = mbar_wait(&bar.ring_full[g % L::kStages0], (g / L::kStages0) & 1, bar.abort_flag,
+                                     status)))
+                    break;
                 tc_fence_after();
                 issue_s(g);
-                // Order per step m: dP^T(m), dV(m) once P^T(m) is stored, S^T(m+1) once
-                // the element-wise warps have loaded P^T(m) (it overwrites those
-                // columns; dV(m), issued before it, reads them first), dK(m) once
-                // dS^T(m) is stored.  The S^T of the next step so runs while dS^T is
-                // formed.  dP^T(m+1) overwrites dS^T(m) and follows dK(m).
+                if (!(ok = mbar_wait(&bar.ring1_full[g & 1], (g >> 1) & 1, bar.abort_flag, status))) break;
+                tc_fence_after();
+                issue_dp(g);
+                // the item's last products that read K and V (its last S^T and dP^T)
+                // are issued: the next item's K and V may load while the rest runs
+                if (n_steps == 1) mma_commit(bar.fixed_empty);
+                // Order per step m: S^T(m+1) as soon as the element-wise warps have
+                // loaded S^T(m) (P^T and dS^T go to the dP^T columns, so the S^T
+                // columns are free and the next S^T runs while P^T(m) is formed), then
+                // dV(m) and dK(m) once P^T(m) and dS^T(m) are stored, then dP^T(m+1),
+                // which overwrites them.
                 for (int n = 0; n < n_steps && ok; ++n) {
                     const uint32_t m = g + n;
-                    const int st = m & 1;
-                    const uint32_t ring = (st * L::kTile) >> 4;
-                    // dP^T = V dout^T (K-major operands, K = D)
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = ((kk >> 2) * T::kChunkBytes + (kk & 3) * 32) >> 4;
-                        mma_ss_lh<idesc_ss>(tmem + kDP, static_cast<uint32_t>(dv_) + off, hi_k,
-                                            static_cast<uint32_t>(dd_k) + ring + off, hi_k, kk > 0 ? 1u : 0u);
+                    const int sq = static_cast<int>(m % L::kStages0), sd = m & 1;
+                    const uint32_t ring_q = (sq * L::kTile) >> 4, ring_d = (sd * L::kTile) >> 4;
+                    if (n + 1 < n_steps) {
+                        if (!(ok = mbar_wait(&bar.ring_full[(m + 1) % L::kStages0], ((m + 1) / L::kStages0) & 1,
+                                             bar.abort_flag, status)))
+                            break;
+                        if (!(ok = mbar_wait(bar.p_read, m & 1, bar.abort_flag, status))) break;
+                        tc_fence_after();
+                        issue_s(m + 1);
                     }
-                    mma_commit(bar.dp_full);
-                    // the item's last products that read K and V (its last S^T and dP^T)
-                    // are issued: the next item's K and V may load while this step's
-                    // dV and dK run
-                    if (n + 1 == n_steps) mma_commit(bar.fixed_empty);
-                    if (!(ok = mbar_wait(bar.p_ready, m & 1, bar.abort_flag, status))) break;
+                    if (!(ok = mbar_wait(bar.ds_ready, m & 1, bar.abort_flag, status))) break;
                     // the first dV of an item overwrites the accumulators: the previous
                     // item's must have been read out
                     if (n == 0 && acc_n > 0 &&
                         !(ok = mbar_wait(bar.acc_free, (acc_n - 1) & 1, bar.abort_flag, status)))
                         break;
                     tc_fence_after();
-                    // dV += P^T dout (A from tensor memory, B MN-major, K = 128 query rows)
+                    // dV += P^T dout and dK += dS^T Q (A from tensor memory: P^T at
+                    // kDP + bwd_kcol, dS^T 32 columns on; B MN-major, K = 128 query rows)
 #pragma unroll
                     for (int kk = 0; kk < kBlockM / 16; ++kk)
-                        mma_ts_lh<idesc_ts>(tmem + kDV, tmem + kS + bwd_kcol(kk),
-                                            static_cast<uint32_t>(dd_mn) + ring + ((kk * 16 * 128) >> 4), hi_mn,
+                        mma_ts_lh<idesc_ts>(tmem + kDV, tmem + kDP + bwd_kcol(kk),
+                                            static_cast<uint32_t>(dd_mn) + ring_d + ((kk * 16 * 128) >> 4), hi_mn,
                                             (n > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < kBlockM / 16; ++kk)
+                        mma_ts_lh<idesc_ts>(tmem + kDK, tmem + kDP + 32 + bwd_kcol(kk),
+                                            static_cast<uint32_t>(dq_mn) + ring_q + ((kk * 16 * 128) >> 4), hi_mn,
+                                            (n > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&bar.ring_empty[sq]);
+                    mma_commit(&bar.ring1_empty[sd]);
                     if (n + 1 < n_steps) {
-                        if (!(ok = mbar_wait(&bar.ring_full[(m + 1) & 1], ((m + 1) >> 1) & 1, bar.abort_flag,
+                        if (!(ok = mbar_wait(&bar.ring1_full[(m + 1) & 1], ((m + 1) >> 1) & 1, bar.abort_flag,
                                              status)))
                             break;
-                        if (!(ok = mbar_wait(bar.p_read, m & 1, bar.abort_flag, status))) break;
                         tc_fence_after();
-                        issue_s(m + 1);
+                        issue_dp(m + 1);
+                        if (n + 2 == n_steps) mma_commit(bar.fixed_empty);
                     }
-                    // dK += dS^T Q
-                    if (!(ok = mbar_wait(bar.ds_ready, m & 1, bar.abort_flag, status))) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < kBlockM / 16; ++kk)
-                        mma_ts_lh<idesc_ts>(tmem + kDK, tmem + kDP + bwd_kcol(kk),
-                                            static_cast<uint32_t>(dq_mn) + ring + ((kk * 16 * 128) >> 4), hi_mn,
-                                            (n > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(&bar.ring_empty[st]);
                 }
                 if (!ok) break;
                 mma_commit(bar.acc_done);
@@ -511,9 +544,8 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                 const int qt = qt0 + n % n_qt;
                 if (!(ok = mbar_wait_warp(bar.s_full, m & 1, bar.abort_flag, status))) break;
                 // the producer's stores of this step's logsumexp and Delta rows are
-                // released by its arrival on ring_full (already complete: the MMA
-                // warp waited for it before the products this wait observed)
-                if (!(ok = mbar_wait_warp(&bar.ring_full[st], (m >> 1) & 1, bar.abort_flag, status))) break;
+                // released by its arrival with the dout tile on ring1_full
+                if (!(ok = mbar_wait_warp(&bar.ring1_full[st], (m >> 1) & 1, bar.abort_flag, status))) break;
                 tc_fence_after();
                 const float* nl2 = lse_s + st * kBlockM;  // -lse * log2(e) per query column
                 const float* ndl = dlt_s + st * kBlockM;  // -Delta per query column
@@ -524,16 +556,20 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                 const bool full = __all_sync(0xffffffffu, i_span != 0u && i_base <= i0 &&
                                                               i0 + 63 <= i_base + static_cast<int>(i_span));
                 // P^T = exp2(s * log2(e) / sqrt(D) - lse * log2(e)) on visible pairs, as
-                // bf16 at bwd_pcol(c); the second chunk's load is in flight while the
-                // first is computed
+                // bf16 pairs kept in registers until dP^T has been read
+                uint32_t pk[2][16];
                 {
                     uint32_t sbuf[2][32];
                     tmem_ld32(tmem + lane_addr + kS + ch * 64, sbuf[0]);
+                    tmem_ld32(tmem + lane_addr + kS + ch * 64 + 32, sbuf[1]);
+                    tmem_wait_ld();
+                    // every S^T value of this warp is in registers: the next S^T may land
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar.p_read);
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         const int c = 2 * ch + cc;
-                        tmem_wait_ld();
-                        if (cc == 0) tmem_ld32(tmem + lane_addr + kS + ch * 64 + 32, sbuf[1]);
                         const uint32_t* sr = sbuf[cc];
                         // scale and shift as packed pairs, then the mask (only on tiles
                         // where some pair of this warp is not visible)
@@ -557,39 +593,25 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                                 pv[e] = static_cast<unsigned>(i - i_base) <= i_span ? pv[e] : 0.f;
                             }
                         }
-                        uint32_t pk[16];
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) pk[e / 2] = pack_bf16x2(pv[e], pv[e + 1]);
-                        tmem_st16(tmem + lane_addr + kS + bwd_pcol(c), pk);
+                        for (int e = 0; e < 32; e += 2) pk[cc][e / 2] = pack_bf16x2(pv[e], pv[e + 1]);
                     }
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar.p_ready);
-                // dS^T = P^T (dP^T - Delta) from the stored bf16 P^T, as bf16 at
-                // kDP + bwd_pcol(c)
+                // dS^T = P^T (dP^T - Delta) from the bf16 P^T; then P^T at kDP +
+                // bwd_pcol(c) and dS^T 32 columns on, over dP^T columns this warp has
+                // read
                 if (!(ok = mbar_wait_warp(bar.dp_full, m & 1, bar.abort_flag, status))) break;
                 tc_fence_after();
                 {
-                    uint32_t dbuf[2][32], pbuf[2][16];
+                    uint32_t dbuf[2][32];
                     tmem_ld32(tmem + lane_addr + kDP + ch * 64, dbuf[0]);
-                    tmem_ld16(tmem + lane_addr + kS + bwd_pcol(2 * ch), pbuf[0]);
+                    tmem_ld32(tmem + lane_addr + kDP + ch * 64 + 32, dbuf[1]);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         const int c = 2 * ch + cc;
-                        tmem_wait_ld();
-                        if (cc == 0) {
-                            tmem_ld32(tmem + lane_addr + kDP + ch * 64 + 32, dbuf[1]);
-                            tmem_ld16(tmem + lane_addr + kS + bwd_pcol(c + 1), pbuf[1]);
-                        } else {
-                            // every P^T value of this warp is in registers: the next S^T may land
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(bar.p_read);
-                        }
                         const uint32_t* dr = dbuf[cc];
-                        const uint32_t* pr = pbuf[cc];
+                        const uint32_t* pr = pk[cc];
                         // dS = P (dP - Delta) on packed pairs; a masked pair has P = 0 and a
                         // finite dP - Delta (rows past the sequence stage Delta = 0), so it
                         // stays 0
@@ -609,7 +631,8 @@ bwd_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
                             dk16[e / 2] = pack_bf16x2(ds[0], ds[1]);
                             dk16[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
                         }
-                        tmem_st16(tmem + lane_addr + kDP + bwd_pcol(c), dk16);
+                        tmem_st16(tmem + lane_addr + kDP + bwd_pcol(c), pk[cc]);
+                        tmem_st16(tmem + lane_addr + kDP + bwd_pcol(c) + 32, dk16);
                     }
                 }
                 tmem_wait_st();
@@ -649,6 +672,12 @@ bwd_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
+    if constexpr (L::kNeedsAlignedBase) {
+        if (smem != smem_raw) {  // uniform across the CTA: every thread leaves here
+            if (threadIdx.x == 0) atomicOr(&g_va_status, kStatusSmemAlign);
+            return;
+        }
+    }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const BwdBars bar = bwd_setup<D, true>(smem, warp);
     const uint32_t tmem = *bar.tmem_slot;

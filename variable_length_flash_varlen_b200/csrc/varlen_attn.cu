@@ -1096,6 +1096,9 @@ int varlen_attention_sync_status(void* stream_, unsigned* status, int clear) {
     *status = word;
     if (word & va::kStatusWaitTimeout)
         return fail(VA_ERR_DEVICE_TIMEOUT, "a bounded wait inside a kernel gave up (status 0x%x)", word);
+    if (word & va::kStatusSmemAlign)
+        return fail(VA_ERR_CUDA, "a kernel's dynamic shared memory was not 1024-byte aligned; it did nothing "
+                                 "(status 0x%x)", word);
     if (word & va::kStatusScheduleOverflow)
         return fail(VA_ERR_INVALID_ARG,
                     "more query blocks than max_seqlen_q allows for: a query length exceeds "
