@@ -40,6 +40,10 @@
 
 namespace va {
 
+// Status bit of the backward kernels (next to the bits of ptx.cuh): a kernel
+// whose layout needs a 1024-byte-aligned shared-memory base found it misaligned.
+constexpr unsigned kStatusSmemAlign = 4u;
+
 constexpr int kBwdThreads = 320;
 constexpr int kBwdEwWarps = 8;
 constexpr int kBwdLoadWarp = 8;

@@ -12,7 +12,6 @@ namespace va {
 enum : unsigned {
     kStatusWaitTimeout = 1u,       // a bounded barrier wait gave up
     kStatusScheduleOverflow = 2u,  // more query tiles than max_seqlen_q allows for
-    kStatusSmemAlign = 4u,         // a kernel's dynamic shared memory was not 1024-byte aligned
 };
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
