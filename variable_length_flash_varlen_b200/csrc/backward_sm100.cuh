@@ -25,11 +25,14 @@
 //                      columns, then dV += P^T dout and dK += dS^T Q (TS form),
 //                      the two accumulators in tensor memory over the whole
 //                      loop; the next S^T runs as soon as S^T has been read
-// An item's resident tiles are reloaded once its last products that read them
-// (its last S and dP, issued first in its last step) are done, its
-// accumulators read out by the element-wise warps before the next item's
-// first product overwrites them; the products of one item's steps
-// and the barrier phases run on across items.
+// The streamed tiles come through two rings: ring 0 (K for dQ, Q for dK/dV,
+// three stages: its last reader ends a step, the next-but-one step's first
+// product starts the next) and ring 1 (V, or dout with its step's lse and
+// Delta, two stages).  An item's resident tiles are reloaded once its last
+// products that read them (its last S and dP) are done, its accumulators read
+// out by the element-wise warps before the next item's first product
+// overwrites them; the products of one item's steps and the barrier phases run
+// on across items.
 // Warp roles (320 threads): warps 0-7 the element-wise work and the epilogue
 // (one key row, or one query row, per thread; warps w and w + 4 share a
 // tensor-memory lane quarter and take one half of the 128 columns each), warp
