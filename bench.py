@@ -273,7 +273,8 @@ def run_reference(args, world, rank):
 
 
 def time_device_steps(fn, steps, warmup, flush_buf, world, stream):
-    """Per-step CUDA-event time of fn() (L2 flushed before each step, outside the events)."""
+    """Per-step CUDA-event time of fn() (L2 flushed before each step, outside the
+    events), the whole loop's time, and the library kernels launched in it."""
     for _ in range(warmup):
         flush_buf.zero_()
         fn()
@@ -283,6 +284,7 @@ def time_device_steps(fn, steps, warmup, flush_buf, world, stream):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     outer0, outer1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = binding.launch_count()
     outer0.record(stream)
     for i in range(steps):
         flush_buf.zero_()
@@ -290,11 +292,12 @@ def time_device_steps(fn, steps, warmup, flush_buf, world, stream):
         fn()
         ends[i].record(stream)
     outer1.record(stream)
+    launches = binding.launch_count() - launches0
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    return step_ms, outer0.elapsed_time(outer1)
+    return step_ms, outer0.elapsed_time(outer1), launches
 
 
 def run_profile_target(args, local):
@@ -385,8 +388,11 @@ def run_ours(args, world, rank, local):
     # clocks are sampled across all timed loops
     clk = ClockSampler(smi_index if not args.no_clock_sampler else None).__enter__()
 
-    def timed(fn):
-        ms, _ = time_device_steps(fn, args.steps, args.warmup, flush, world, stream)
+    launches = {}
+
+    def timed(fn, leg):
+        ms, _, n = time_device_steps(fn, args.steps, args.warmup, flush, world, stream)
+        launches[leg] = n
         local_s = sum(ms) / 1e3
         return ms, local_s, max_over_ranks(local_s, world)
 
@@ -396,7 +402,7 @@ def run_ours(args, world, rank, local):
         out = torch.empty_like(d[0])
         lse = torch.empty(wl.total_q, wl.H, dtype=torch.float32, device=dev)
         flops = accounting.attention_flops(wl)
-        ms, local_s, max_s = timed(_fwd_call(wl, d, out, lse))
+        ms, local_s, max_s = timed(_fwd_call(wl, d, out, lse), name)
         value = sum_over_ranks(flops * args.steps, world) / max_s / 1e12
         achieved = flops / (local_s / args.steps) / 1e12
         return wl, host, d, (out, lse), {
@@ -405,7 +411,7 @@ def run_ours(args, world, rank, local):
             "roofline": _tensor_roofline(achieved, peak, pk,
                                          kernel=f"prefill_fwd_kernel<{wl.D}> (+ schedule build, same call)",
                                          traffic=recorded_traffic("prefill_fwd_kernel", name)),
-            "gpu_launches": 2 * args.steps}, ms
+            "gpu_launches": launches[name]}, ms
 
     # ---- the headline: prefill TFLOP/s on the largest configuration (sliding window)
     wl, host, d, (out, lse), head, step_ms = prefill_leg(args.workload)
@@ -424,7 +430,7 @@ def run_ours(args, world, rank, local):
     _, dd = _inputs_on(dwl, dev)
     outd = torch.empty_like(dd[0])
     lsed = torch.empty(dwl.total_q, dwl.H, dtype=torch.float32, device=dev)
-    _, d_local, d_max = timed(_fwd_call(dwl, dd, outd, lsed))
+    _, d_local, d_max = timed(_fwd_call(dwl, dd, outd, lsed), "decode")
     dbytes = accounting.decode_bytes(dwl)
     d_value = sum_over_ranks(dbytes * args.steps, world) / d_max / 1e9
     del dd, outd, lsed
@@ -447,7 +453,7 @@ def run_ours(args, world, rank, local):
                                          fwl.window, fsc["q_scale"], fsc["k_scale"], fsc["v_scale"],
                                          fsc["o_scale"], out=fout, lse=flse)
 
-    _, _, f_max = timed(fstep)
+    _, _, f_max = timed(fstep, "fp8")
     fflops = accounting.attention_flops(fwl)
     f_value = sum_over_ranks(fflops * args.steps, world) / f_max / 1e12
     # E4M3 dense tensor peak: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
@@ -472,7 +478,7 @@ def run_ours(args, world, rank, local):
                                          bwl.H_kv, bwl.max_seqlen_q, bwl.max_seqlen_k, bwl.D,
                                          bwl.causal, bwl.window, dq=gq, dk=gk, dv=gv)
 
-        _, _, b_max = timed(bstep)
+        _, _, b_max = timed(bstep, "bwd:" + name)
         bflops = accounting.backward_flops(bwl)
         b_value = sum_over_ranks(bflops * args.steps, world) / b_max / 1e12
         backward[name] = {
@@ -480,7 +486,7 @@ def run_ours(args, world, rank, local):
             "ms_per_step": b_max / args.steps * 1e3, "flops_per_step_per_gpu": bflops,
             "roofline": _tensor_roofline(b_value / world, peak, pk,
                                          kernel="bwd_dq_kernel + bwd_dkdv_kernel (same call)"),
-            "gpu_launches": 2 * args.steps}
+            "gpu_launches": launches["bwd:" + name]}
         del bd, bq, bk, bv, ddo, bout, blse, gq, gk, gv
 
     # ---- end to end on the headline workload through the host-buffer entry point
@@ -497,7 +503,7 @@ def run_ours(args, world, rank, local):
                                           wl.max_seqlen_q, wl.max_seqlen_k, wl.D, wl.causal,
                                           wl.window, outh, lseh)
 
-    _, _, e_max = timed(estep)
+    _, _, e_max = timed(estep, "e2e")
     clk.__exit__(None, None, None)
     flops = head["flops_per_step_per_gpu"]
     e_value = sum_over_ranks(flops * args.steps, world) / e_max / 1e12
@@ -536,7 +542,7 @@ def run_ours(args, world, rank, local):
                                 "peak_kind": f"{peak_kind} copy",
                                 "kernel": "decode_stream_kernel<128> (+ combine and counter reset, same call)",
                                 "traffic": recorded_traffic("decode_stream_kernel", "decode")},
-                   "gpu_launches": 2 * args.steps},
+                   "gpu_launches": launches["decode"]},
         "chunked_prefill": chunked,
         "fp8": {"workload": "mha_noncausal", "entry": "varlen_attention_fwd_fp8", "dtype": "e4m3",
                 "scales": fsc, "value": f_value, "unit": "TFLOP/s",
@@ -545,12 +551,12 @@ def run_ours(args, world, rank, local):
                              "unit": "TFLOP/s", "frac": f_value / world / fp8_peak,
                              "peak_kind": f"{peak_kind} bf16 burst x 2 (nominal e4m3 / bf16 ratio)",
                              "kernel": "prefill_fwd_kernel<128, E4M3> (+ schedule build, same call)"},
-                "gpu_launches": 2 * args.steps},
+                "gpu_launches": launches["fp8"]},
         "backward": backward,
         "e2e": {"value": e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "entry": "varlen_attention_fwd_host",
-                "workload": args.workload},
-        "gpu_launches": 2 * args.steps,
+                "workload": args.workload, "gpu_launches": launches["e2e"]},
+        "gpu_launches": launches[args.workload],
         "clocks": clocks,
         "cpu_baseline": cpu,
         "step_ms": [round(x, 4) for x in step_ms],

@@ -327,6 +327,15 @@ const char* varlen_attention_last_error(void);
 /* Library ABI version (major * 100 + minor). */
 int varlen_attention_version(void);
 
+/*
+ * Diagnostic: the number of kernels this library has launched in this process
+ * so far (every device and host thread; a bf16 prefill call counts its schedule
+ * build and its two tile-kernel launches, an E4M3 call two, a decode call two,
+ * a backward call four).  The difference across a timed region is the number
+ * of the library's kernels launched in it.  Never fails.
+ */
+unsigned long long varlen_attention_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

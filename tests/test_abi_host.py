@@ -139,3 +139,10 @@ def test_host_entry_rejects_bad_host_cu_seqlens_before_device_work(lib, cq, ck, 
 def test_sync_status_rejects_null_pointer(lib):
     assert lib.varlen_attention_sync_status(None, None, 0) == -1
     assert b"status is NULL" in lib.varlen_attention_last_error()
+
+
+def test_launch_count_is_a_plain_counter(lib):
+    # no device work is needed to read it; nothing was launched by these host-only tests
+    lib.varlen_attention_launch_count.restype = ctypes.c_ulonglong
+    n = lib.varlen_attention_launch_count()
+    assert n == lib.varlen_attention_launch_count()

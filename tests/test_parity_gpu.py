@@ -346,3 +346,38 @@ def test_full_size_sampled_rows(oracle_lib, name):
     compare(out, lse, ref_o, ref_l, rows=rows)
     # every row written: no NaN left from the NaN-filled output buffers
     assert not torch.isnan(out).any() and not torch.isnan(lse).any()
+
+
+# --- launch counts (the bench reports the counter's difference over its timed loops) ----------
+
+def test_launch_counter_counts_each_entry_points_kernels():
+    def launched(fn):
+        n0 = binding.launch_count()
+        fn()
+        torch.cuda.synchronize()
+        return binding.launch_count() - n0
+
+    wl = workloads.named("worked_example")  # bf16 prefill: schedule build, residual and main variant
+    q, k, v = workloads.make_qkv(wl)
+    dev = to_device_inputs(wl, q, k, v)
+    assert launched(lambda: run_gpu(wl, q, k, v, dev_inputs=dev)) == 3
+    out, lse = run_gpu(wl, q, k, v, dev_inputs=dev)
+    dq_, dk_, dv_, cq, ck = dev
+    do = torch.randn_like(dq_)
+    # backward: two list builds, dQ, dK/dV
+    assert launched(lambda: binding.varlen_attention_bwd(do, dq_, dk_, dv_, out, lse, cq, ck, wl.batch, wl.H,
+                                                         wl.H_kv, wl.max_seqlen_q, wl.max_seqlen_k, wl.D,
+                                                         wl.causal, wl.window)) == 4
+    dwl = workloads.named("decode", scale=1 / 32)  # decode: stream and combine
+    qd, kd, vd = workloads.make_qkv(dwl)
+    ddev = to_device_inputs(dwl, qd, kd, vd)
+    assert launched(lambda: run_gpu(dwl, qd, kd, vd, dev_inputs=ddev)) == 2
+    fwl = workloads.named("mha_noncausal", scale=0.1)  # E4M3: schedule build and the one variant
+    q8, k8, v8, sc = workloads.make_qkv_fp8(fwl)
+    fcq = torch.tensor(fwl.cu_q, dtype=torch.int32, device="cuda")
+    fck = torch.tensor(fwl.cu_k, dtype=torch.int32, device="cuda")
+    q8d, k8d, v8d = q8.cuda(), k8.cuda(), v8.cuda()
+    assert launched(lambda: binding.varlen_attention_fwd_fp8(
+        q8d, k8d, v8d, fcq, fck, fwl.batch, fwl.H, fwl.H_kv, fwl.max_seqlen_q, fwl.max_seqlen_k, fwl.D,
+        fwl.causal, fwl.window, sc["q_scale"], sc["k_scale"], sc["v_scale"], sc["o_scale"])) == 2
+    assert binding.device_status(clear=True) == 0

@@ -42,6 +42,7 @@ SIGNATURES = {
     "varlen_attention_selftest_wait_timeout": (_I, [_P, _P]),
     "varlen_attention_last_error": (ctypes.c_char_p, []),
     "varlen_attention_version": (_I, []),
+    "varlen_attention_launch_count": (ctypes.c_ulonglong, []),
 }
 
 _lib = None
@@ -322,6 +323,11 @@ def host_chunks(cu_seqlens_q, cu_seqlens_k, batch: int, causal: bool, window: in
     _check(lib.varlen_attention_host_chunks(cq.data_ptr(), ck.data_ptr(), batch, int(causal), window,
                                             input_bytes, buf, n.value, ctypes.byref(n)))
     return [dict(zip(HOST_CHUNK_FIELDS, buf[9 * c: 9 * c + 9])) for c in range(n.value)]
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process so far (a diagnostic)."""
+    return int(load().varlen_attention_launch_count())
 
 
 def device_status(clear: bool = True) -> int:

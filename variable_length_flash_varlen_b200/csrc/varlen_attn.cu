@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdarg>
@@ -61,6 +62,11 @@ int cuda_fail(cudaError_t e, const char* what) {
     } while (0)
 
 constexpr int kMaxDevices = 64;
+
+// Kernels this library has launched in this process (every device and thread):
+// a diagnostic for counting the launches of a timed region.
+std::atomic<unsigned long long> g_launches{0};
+void note_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 // Host-buffer entry point: up to this many pipelined chunks, once the inputs
 // reach this size.
 constexpr int kHostChunks = 16;
@@ -324,6 +330,7 @@ cudaError_t launch_prefill(const Args& a, const va::PrefillMaps& maps, const va:
     cfg.numAttrs = 1;
     if (a.fp8) {
         cfg.dynamicSmemBytes = va::PrefillSmem<128, va::ElemE4m3>::kAlloc;
+        note_launches(1);
         return cudaLaunchKernelEx(&cfg, va::prefill_fwd_kernel<128, va::ElemE4m3, false>, maps, p);
     }
     // bf16: the residual variant over the list's few-key part first (its CTAs
@@ -331,6 +338,7 @@ cudaError_t launch_prefill(const Args& a, const va::PrefillMaps& maps, const va:
     // part as its programmatic dependent, on the SMs the residual one leaves
     va::PrefillParams pm = p;
     pm.after_residual = 1;
+    note_launches(2);
     cudaError_t e;
     if (a.D == 64) {
         cfg.dynamicSmemBytes = va::PrefillSmem<64, va::ElemBf16>::kAlloc;
@@ -367,6 +375,7 @@ int run_prefill(const Args& a, const DeviceInfo& dev, cudaStream_t stream) {
         return rc;
     }
 
+    note_launches(1);
     va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
         a.cu_q, a.cu_k, a.seqused_k, a.batch, a.causal, a.window, a.fp8 ? 0 : 1, cap, key_slots,
         scratch, tiles, hdr);
@@ -450,9 +459,11 @@ int run_decode(const Args& a, const DeviceInfo& dev, int split_keys, cudaStream_
     p.lse = a.lse;
     const int grid = static_cast<int>(std::min<long long>(dev.num_sms, n_units));
     if (a.D == 64) {
+        note_launches(2);
         va::decode_stream_kernel<64><<<grid, va::kDecodeThreads, va::DecodeSmem<64>::kAlloc, stream>>>(tk, tv, tk8, tv8, p);
         va::decode_combine_kernel<64><<<a.batch * a.H, 64, 0, stream>>>(p);
     } else {
+        note_launches(2);
         va::decode_stream_kernel<128><<<grid, va::kDecodeThreads, va::DecodeSmem<128>::kAlloc, stream>>>(tk, tv, tk8, tv8, p);
         va::decode_combine_kernel<128><<<a.batch * a.H, 128, 0, stream>>>(p);
     }
@@ -552,6 +563,7 @@ int run_backward(const BwdArgs& g, cudaStream_t stream) {
         return s;
     };
     if (cap_q > 0)
+        note_launches(2);
         va::build_bwd_list_kernel<<<1, va::kBuildThreads, slots(cap_q) * 8, stream>>>(
             a.cu_q, a.cu_k, a.batch, a.causal, a.window, 0, cap_q, slots(cap_q), scratch_q, list_q, hdr_q);
     if (cap_k > 0)
@@ -589,6 +601,7 @@ int run_backward(const BwdArgs& g, cudaStream_t stream) {
     // dK/dV kernel reads
     const int grid_q = static_cast<int>(std::min<long long>(info->num_sms, cap_q_ll * a.H));
     const int grid_kv = static_cast<int>(std::min<long long>(info->num_sms, cap_k_ll * a.H_kv));
+    note_launches((grid_q > 0) + (grid_kv > 0));
     if (a.D == 64) {
         if (grid_q > 0) va::bwd_dq_kernel<64><<<grid_q, va::kBwdThreads, va::BwdSmem<64, true>::kAlloc, stream>>>(maps, p);
         if (grid_kv > 0)
@@ -694,6 +707,7 @@ int run_prefill_noalloc(const Args& a, cudaStream_t stream) {
     if ((rc = make_prefill_maps(a, &maps)) != VA_OK) return rc;
     // the builder rewrites the whole header (count and work counter) and every
     // list entry it hands out, so nothing left by the previous call is read
+    note_launches(1);
     va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
         a.cu_q, a.cu_k, a.seqused_k, a.batch, a.causal, a.window, a.fp8 ? 0 : 1, cap, key_slots,
         scratch, tiles, hdr);
@@ -1037,6 +1051,7 @@ int varlen_attention_schedule(const int32_t* cu_seqlens_q, const int32_t* cu_seq
     const size_t list_bytes = static_cast<size_t>(capacity) * sizeof(va::TileEntry);
     VA_CUDA(ws_alloc(reinterpret_cast<void**>(&ws), 256 + list_bytes, stream));
     auto* hdr = reinterpret_cast<va::SchedHeader*>(ws);
+    note_launches(1);
     va::build_schedule_kernel<<<1, va::kBuildThreads, key_slots * 8, stream>>>(
         cu_seqlens_q, cu_seqlens_k, nullptr, batch, causal ? 1 : 0, window, 1, capacity, key_slots,
         reinterpret_cast<va::TileEntry*>(ws + 256), reinterpret_cast<va::TileEntry*>(tiles), hdr);
@@ -1123,6 +1138,7 @@ int varlen_attention_fwd_noalloc(const void* q, const void* k, const void* v,
 int varlen_attention_selftest_wait_timeout(int32_t* gave_up, void* stream) {
     g_last_error[0] = 0;
     if (!gave_up) return fail(VA_ERR_INVALID_ARG, "gave_up is NULL");
+    note_launches(1);
     va::wait_timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(gave_up);
     VA_CUDA(cudaGetLastError());
     return VA_OK;
@@ -1131,5 +1147,7 @@ int varlen_attention_selftest_wait_timeout(int32_t* gave_up, void* stream) {
 const char* varlen_attention_last_error(void) { return g_last_error; }
 
 int varlen_attention_version(void) { return 100; }
+
+unsigned long long varlen_attention_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"
